@@ -313,6 +313,22 @@ def qkv(cfg: Config, W: Dict, x: np.ndarray, angles: np.ndarray, dtype=np.float6
     return rope_rotate(q, angles), rope_rotate(k, angles), v.reshape(S, nkv, hd)
 
 
+def o_residual(W: Dict, o: np.ndarray, x: np.ndarray, dtype=np.float64) -> np.ndarray:
+    """h = x + o W_o^T: the o-projection and the attention residual (o: [S, nh*hd])."""
+    return x + o @ _np(W["wo"], dtype).T
+
+
+def ffn_act(cfg: Config, W: Dict, h: np.ndarray, dtype=np.float64) -> np.ndarray:
+    """a = silu(hn W_g^T) * (hn W_u^T), hn = RMSNorm(h, ffn_norm)."""
+    hn = rms_norm(h, _np(W["ffn_norm"], dtype), cfg.rms_eps)
+    return silu(hn @ _np(W["wg"], dtype).T) * (hn @ _np(W["wu"], dtype).T)
+
+
+def down_residual(W: Dict, a: np.ndarray, h: np.ndarray, dtype=np.float64) -> np.ndarray:
+    """x' = h + a W_down^T (before any DeepStack add)."""
+    return h + a @ _np(W["wd"], dtype).T
+
+
 def layer(cfg: Config, W: Dict, x, pos: np.ndarray, ds_slab=None, ds_rows=None,
           dtype=np.float64, rows: Optional[np.ndarray] = None,
           taps: Optional[Dict] = None) -> np.ndarray:
@@ -333,13 +349,10 @@ def layer(cfg: Config, W: Dict, x, pos: np.ndarray, ds_slab=None, ds_rows=None,
     o = attention(q, k, v, rows)
     sel = np.arange(S) if rows is None else np.asarray(rows)
     h = np.zeros_like(x)
-    h[sel] = x[sel] + o[sel].reshape(len(sel), nh * hd) @ _np(W["wo"], dtype).T
-    hn = rms_norm(h[sel], _np(W["ffn_norm"], dtype), cfg.rms_eps)
-    g = hn @ _np(W["wg"], dtype).T
-    u = hn @ _np(W["wu"], dtype).T
-    a = silu(g) * u
+    h[sel] = o_residual(W, o[sel].reshape(len(sel), nh * hd), x[sel], dtype)
+    a = ffn_act(cfg, W, h[sel], dtype)
     out = np.zeros_like(x)
-    out[sel] = h[sel] + a @ _np(W["wd"], dtype).T
+    out[sel] = down_residual(W, a, h[sel], dtype)
     if ds_slab is not None:
         slab = _np(ds_slab, dtype)
         ds_rows = np.asarray(ds_rows)

@@ -1,0 +1,300 @@
+// Causal GQA flash attention on tcgen05 tensor cores (sm_100a), head_dim 128.
+//
+// o[p, h] = sum_{j <= p} softmax_j(q_p,h . k_j,g / sqrt(128)) v_j,g with
+// g = h / (nh / nkv) (cortiq qwen3te.rs, the per-pair loop and
+// `Qwen3Encoder::attention_gemm`), computed with an online softmax so no
+// S x S matrix exists.
+//
+// One CTA = one 128-row query tile of one head; CTAs are ordered longest
+// (last query tile) first, and the query heads of one KV group are
+// neighbours so their K/V tiles are shared through L2. Causality skips every
+// key tile past the diagonal; the diagonal tile is masked in registers.
+//
+// Roles (192 threads):
+//   warp 0    one thread: TMA loads of Q (once), K and V tiles (two-stage
+//             rings), 128-byte swizzled.
+//   warp 1    one thread: S_j = Q K_j^T into one of two TMEM buffers, and
+//             O += P_j V_j into the TMEM accumulator (V as an MN-major
+//             operand, no transpose pass).
+//   warps 2-5 softmax: thread = query row; reads S_j with tcgen05.ld, keeps
+//             the running max m and sum l in registers, rescales O in TMEM
+//             when m grows, writes P_j (bf16) to shared memory in the
+//             swizzled K-major layout the MMA reads, and at the end writes
+//             O / l.
+#include "q3vl_device.cuh"
+#include "q3vl_internal.h"
+
+namespace q3vl {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kTile = 128;               // query rows per CTA and keys per tile
+constexpr int kBlockBytes = 128 * 64 * 2;  // one [128 x 64] bf16 swizzle block
+constexpr int kTileBytes = 2 * kBlockBytes;  // [128 x 128] bf16
+constexpr size_t kSmem = 1024 + 6 * size_t(kTileBytes) + 256;  // Q, K[2], V[2], P
+
+struct Params {
+  int64_t S;
+  int nh, nkv, num_qt;
+  int32_t k_col0, v_col0;
+  __nv_bfloat16* o;
+  int64_t ldo;
+  float scale_log2;  // log2(e) / sqrt(128)
+  int32_t* err;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint8_t* sQ = smem;
+  uint8_t* sK = smem + kTileBytes;      // 2 stages
+  uint8_t* sV = smem + 3 * kTileBytes;  // 2 stages
+  uint8_t* sP = smem + 5 * kTileBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 6 * kTileBytes);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;   // [2]
+  uint64_t* k_empty = bars + 3;  // [2]
+  uint64_t* v_full = bars + 5;   // [2]
+  uint64_t* v_empty = bars + 7;  // [2]
+  uint64_t* s_full = bars + 9;   // [2]
+  uint64_t* p_full = bars + 11;
+  uint64_t* o_done = bars + 12;
+  uint64_t* drain = bars + 13;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = p.num_qt - 1 - static_cast<int>(blockIdx.x / p.nh);
+  const int h = static_cast<int>(blockIdx.x % p.nh);
+  const int g = h / (p.nh / p.nkv);
+  const int n_kv = qt + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(k_full + s, 1); mbar_init(k_empty + s, 1);
+      mbar_init(v_full + s, 1); mbar_init(v_empty + s, 1);
+      mbar_init(s_full + s, 1);
+    }
+    mbar_init(p_full, 128);
+    mbar_init(o_done, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tO = tmem + 256;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, kTileBytes);
+      tma_load_2d(sQ, &tm, q_full, h * 128, qt * kTile);
+      tma_load_2d(sQ + kBlockBytes, &tm, q_full, h * 128 + 64, qt * kTile);
+      int nk_issued = 0, nv_issued = 0;
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        if (!mbar_wait(k_empty + s, ph ^ 1, p.err, kWhereAttnProducer, abort_flag)) break;
+        mbar_arrive_expect_tx(k_full + s, kTileBytes);
+        tma_load_2d(sK + s * kTileBytes, &tm, k_full + s, p.k_col0 + g * 128, j * kTile);
+        tma_load_2d(sK + s * kTileBytes + kBlockBytes, &tm, k_full + s, p.k_col0 + g * 128 + 64,
+                    j * kTile);
+        ++nk_issued;
+        if (!mbar_wait(v_empty + s, ph ^ 1, p.err, kWhereAttnProducer, abort_flag)) break;
+        mbar_arrive_expect_tx(v_full + s, kTileBytes);
+        tma_load_2d(sV + s * kTileBytes, &tm, v_full + s, p.v_col0 + g * 128, j * kTile);
+        tma_load_2d(sV + s * kTileBytes + kBlockBytes, &tm, v_full + s, p.v_col0 + g * 128 + 64,
+                    j * kTile);
+        ++nv_issued;
+      }
+      // Every issued load must land before the block exits: the last two
+      // loads of each ring are the only ones whose completion may be unseen.
+      mbar_wait(q_full, 0, p.err, kWhereAttnDrain, nullptr);
+      for (int j = nk_issued - 2; j < nk_issued; ++j)
+        if (j >= 0) mbar_wait(k_full + (j & 1), (j >> 1) & 1, p.err, kWhereAttnDrain, nullptr);
+      for (int j = nv_issued - 2; j < nv_issued; ++j)
+        if (j >= 0) mbar_wait(v_full + (j & 1), (j >> 1) & 1, p.err, kWhereAttnDrain, nullptr);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, 128, false, true);
+      const uint32_t q0 = smem_u32(sQ), p0 = smem_u32(sP);
+      bool ok = mbar_wait(q_full, 0, p.err, kWhereAttnMma, abort_flag);
+      auto issue_s = [&](int j) -> bool {
+        const int s = j & 1;
+        if (!mbar_wait(k_full + s, (j >> 1) & 1, p.err, kWhereAttnMma, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t k0 = smem_u32(sK + s * kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kBlockBytes + (kk & 3) * 32;
+          umma_bf16_ss(tmem + s * 128, sdesc_sw128(q0 + off, 16, 1024),
+                       sdesc_sw128(k0 + off, 16, 1024), idesc_s, kk > 0);
+        }
+        umma_commit(s_full + s);
+        umma_commit(k_empty + s);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int j = 0; ok && j < n_kv; ++j) {
+        if (j + 1 < n_kv && !issue_s(j + 1)) break;
+        if (!mbar_wait(p_full, j & 1, p.err, kWhereAttnMma, abort_flag)) break;
+        tc_fence_after();
+        const int s = j & 1;
+        if (!mbar_wait(v_full + s, (j >> 1) & 1, p.err, kWhereAttnMma, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t v0 = smem_u32(sV + s * kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          umma_bf16_ss(tO, sdesc_sw128(p0 + (kk >> 2) * kBlockBytes + (kk & 3) * 32, 16, 1024),
+                       sdesc_sw128(v0 + kk * 2048, kBlockBytes, 1024), idesc_o, (j | kk) != 0);
+        }
+        umma_commit(o_done);
+        umma_commit(v_empty + s);
+      }
+      umma_commit(drain);
+      mbar_wait(drain, 0, p.err, kWhereAttnDrain, nullptr);
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_field = static_cast<uint32_t>(quarter * 32) << 16;
+    const int64_t qpos = int64_t(qt) * kTile + r;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      ok = mbar_wait(s_full + (j & 1), (j >> 1) & 1, p.err, kWhereAttnSoftmax, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+      float x[128];
+      {
+        uint32_t raw[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tmem + (j & 1) * 128 + lane_field + 32 * c, raw[c]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int t = 0; t < 32; ++t) x[32 * c + t] = __uint_as_float(raw[c][t]) * p.scale_log2;
+      }
+      if (j == qt) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c > r) x[c] = -INFINITY;
+      }
+      float mx = x[0];
+#pragma unroll
+      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, x[c]);
+      const float m_new = fmaxf(m, mx);
+      const float alpha = exp2f(m - m_new);
+      float rs = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const __nv_bfloat162 b =
+            __floats2bfloat162_rn(exp2f(x[2 * c] - m_new), exp2f(x[2 * c + 1] - m_new));
+        const float2 f = __bfloat1622float2(b);
+        rs += f.x + f.y;
+        pk[c] = *reinterpret_cast<const uint32_t*>(&b);
+      }
+      if (j > 0) {
+        // P_{j-1} V_{j-1} must be done before O is rescaled and P is reused.
+        ok = mbar_wait(o_done, (j - 1) & 1, p.err, kWhereAttnSoftmax, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, m_new > m)) {
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + lane_field + 32 * c, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * alpha);
+            tmem_st32(tO + lane_field + 32 * c, o);
+          }
+          tmem_st_wait();
+        }
+      }
+      l = l * alpha + rs;
+      m = m_new;
+      // P row r, 128-byte swizzle: 16-byte chunk c8 of row r sits at c8 ^ (r % 8).
+#pragma unroll
+      for (int cc = 0; cc < 16; ++cc) {
+        const int off = (cc >> 3) * kBlockBytes + r * 128 + (((cc & 7) ^ (r & 7)) << 4);
+        *reinterpret_cast<uint4*>(sP + off) =
+            make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    if (ok) {
+      ok = mbar_wait(o_done, (n_kv - 1) & 1, p.err, kWhereAttnSoftmax, abort_flag);
+      if (__all_sync(0xffffffffu, ok)) {
+        tc_fence_after();
+        const float inv_l = 1.0f / l;
+        __nv_bfloat16* dst = p.o + qpos * p.ldo + h * 128;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + lane_field + 32 * c, o);
+          tmem_ld_wait();
+          if (qpos < p.S) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+              d4[t] = make_uint4(
+                  pack_bf16x2(__uint_as_float(o[8 * t]) * inv_l, __uint_as_float(o[8 * t + 1]) * inv_l),
+                  pack_bf16x2(__uint_as_float(o[8 * t + 2]) * inv_l, __uint_as_float(o[8 * t + 3]) * inv_l),
+                  pack_bf16x2(__uint_as_float(o[8 * t + 4]) * inv_l, __uint_as_float(o[8 * t + 5]) * inv_l),
+                  pack_bf16x2(__uint_as_float(o[8 * t + 6]) * inv_l, __uint_as_float(o[8 * t + 7]) * inv_l));
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_attention_tc(const q3vl_config& c, const void* qkv, int64_t S, void* o,
+                                cudaStream_t st) {
+  const int64_t Ntot = qkv_dim(c);
+  CUtensorMap tm;
+  if (!make_tmap_bf16(&tm, qkv, S, Ntot, Ntot, 64, 128)) return cudaErrorInvalidValue;
+  Params p;
+  p.S = S;
+  p.nh = c.n_heads;
+  p.nkv = c.n_kv_heads;
+  p.num_qt = static_cast<int>((S + kTile - 1) / kTile);
+  p.k_col0 = static_cast<int32_t>(q_dim(c));
+  p.v_col0 = static_cast<int32_t>(q_dim(c) + kv_dim(c));
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.ldo = q_dim(c);
+  p.scale_log2 = 1.4426950408889634f / sqrtf(128.0f);
+  p.err = device_error_ptr();
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kSmem));
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>(int64_t(p.num_qt) * p.nh);
+  attn_tc_kernel<<<grid, kThreads, kSmem, st>>>(tm, p);
+  return counted_launch(1);
+}
+
+}  // namespace q3vl

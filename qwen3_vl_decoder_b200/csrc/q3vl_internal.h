@@ -1,0 +1,115 @@
+// Host-side internals of libq3vl: workspace layout, kernel launchers and
+// shared helpers. Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "q3vl.h"
+
+namespace q3vl {
+
+constexpr int kHeadDim = 128;
+constexpr int kHalf = kHeadDim / 2;
+
+inline size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+inline int64_t q_dim(const q3vl_config& c) { return int64_t(c.n_heads) * c.head_dim; }
+inline int64_t kv_dim(const q3vl_config& c) { return int64_t(c.n_kv_heads) * c.head_dim; }
+inline int64_t qkv_dim(const q3vl_config& c) { return q_dim(c) + 2 * kv_dim(c); }
+inline size_t elem_bytes(const q3vl_config& c) { return c.dtype == Q3VL_DTYPE_BF16 ? 2 : 4; }
+
+// Offsets (bytes) of every region of the layer workspace.
+struct WsLayout {
+  size_t cos_sin = 0;  // fp32 [S][64][2]
+  size_t inv1 = 0;     // fp32 [S] input-norm inv_rms
+  size_t inv2 = 0;     // fp32 [S] post-attention-norm inv_rms
+  size_t ds_map = 0;   // int32 [S]
+  size_t qkv = 0;      // dtype [S][Ntot]
+  size_t o = 0;        // dtype [S][Dq]
+  size_t h = 0;        // dtype [S][H]
+  size_t act = 0;      // dtype [S][I]
+  size_t total = 0;
+};
+WsLayout ws_layout(const q3vl_config& c, int64_t S);
+
+// Offsets of the packed-layer regions.
+struct PackLayout {
+  size_t w_qkv = 0, b_qkv = 0, q_norm = 0, k_norm = 0, w_o = 0, w_gu = 0, w_down = 0, total = 0;
+};
+PackLayout pack_layout(const q3vl_config& c);
+
+// Per-device error record [code, where] (a __device__ array of 2 int32).
+int32_t* device_error_ptr();
+
+// Thread-local last-error message.
+int set_error(int code, const std::string& msg);
+int cuda_check(cudaError_t e, const char* what);
+
+// Tensor map over a row-major [rows, cols] bf16 matrix with row stride
+// `ld` elements, box (box_cols x box_rows), 128-byte swizzle, zero fill.
+bool make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols,
+                    uint64_t ld, uint32_t box_cols, uint32_t box_rows);
+
+// ---------------------------------------------------------------------------
+// Launchers (all enqueue on `st`, return the launch status).
+// ---------------------------------------------------------------------------
+cudaError_t launch_positions(const uint8_t* tt, int64_t S, const int32_t* grids, int n_grids,
+                             int32_t* pos, int32_t* info, cudaStream_t st);
+cudaError_t launch_rope_table(const q3vl_config& c, const int32_t* pos, int64_t S, float* cs,
+                              cudaStream_t st);
+cudaError_t launch_rowstat(const q3vl_config& c, const void* x, int64_t S, int64_t width,
+                           float* inv, cudaStream_t st);
+cudaError_t launch_final_norm(const q3vl_config& c, void* x, int64_t S, const void* gain,
+                              cudaStream_t st);
+cudaError_t launch_deepstack_map(const int32_t* rows, int n_img, int64_t S, int32_t* map,
+                                 cudaStream_t st);
+cudaError_t launch_pack(const q3vl_config& c, const q3vl_raw_weights& raw, void* packed,
+                        cudaStream_t st);
+cudaError_t launch_selftest_timeout(uint32_t timeout_us, cudaStream_t st);
+
+// bf16 tensor-core path (tcgen05 + TMA).
+enum class Epi : int { kQkv = 0, kResidual = 1, kSwiGLU = 2, kPlain = 3 };
+struct GemmArgs {
+  const void* A;        // [M, K] bf16
+  const void* B;        // [N, K] bf16
+  int64_t M, N, K;
+  void* out;            // bf16; row stride ldo
+  int64_t ldo;
+  const float* row_scale;  // [M] or null (kQkv, kSwiGLU)
+  const float* bias;       // [N] or null (kQkv)
+  const float* q_norm;     // [128] (kQkv)
+  const float* k_norm;     // [128] (kQkv)
+  const float* cos_sin;    // [M][64][2] (kQkv)
+  int64_t q_cols, k_cols;  // column ranges [0,q_cols) = q heads, [q_cols, q_cols+k_cols) = k
+  float eps;
+  const void* resid;       // bf16 [M, ldo] (kResidual)
+  const void* ds_slab;     // bf16 [n_img, N] (kResidual) or null
+  const int32_t* ds_map;   // [M] (kResidual) or null
+};
+cudaError_t launch_gemm_tc(Epi epi, const GemmArgs& a, cudaStream_t st);
+cudaError_t launch_attention_tc(const q3vl_config& c, const void* qkv, int64_t S, void* o,
+                                cudaStream_t st);
+
+// fp32 CUDA-core path.
+cudaError_t launch_gemm_f32(Epi epi, const GemmArgs& a, cudaStream_t st);
+cudaError_t launch_qk_norm_rope_f32(const q3vl_config& c, float* qkv, int64_t S,
+                                    const float* q_norm, const float* k_norm, const float* cs,
+                                    cudaStream_t st);
+cudaError_t launch_gemm_swiglu_f32(const float* A, const float* B, int64_t M, int64_t I, int64_t K,
+                                   const float* row_scale, float* act, cudaStream_t st);
+cudaError_t launch_attention_f32(const q3vl_config& c, const float* qkv, int64_t S, float* o,
+                                 cudaStream_t st);
+
+// Device count of SMs (cached per device).
+int sm_count();
+
+// Adds n to the process-wide count of kernels this library enqueued and
+// returns the launch status of the last one.
+cudaError_t counted_launch(int n);
+
+}  // namespace q3vl

@@ -1,0 +1,128 @@
+"""The C-ABI library loads and exports every symbol the header declares (no GPU).
+
+Only host-side paths are exercised here: size queries and argument
+validation, which return before any CUDA call.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "q3vl.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from qwen3_vl_decoder_b200 import build
+    build.build()
+    from qwen3_vl_decoder_b200 import _abi
+    return _abi.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(q3vl_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_three_north_calls():
+    names = declared_functions()
+    for n in ("q3vl_mrope_positions", "q3vl_layer_prefill", "q3vl_stack_prefill"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_binding_covers_every_declared_symbol():
+    from qwen3_vl_decoder_b200 import _abi
+    assert set(declared_functions()) == set(_abi.SIGNATURES)
+
+
+def _cfg(**kw):
+    from qwen3_vl_decoder_b200 import config
+    base = dict(hidden=2560, n_heads=32, n_kv_heads=8, intermediate=9728, dtype="bf16",
+                qkv_bias=True)
+    base.update(kw)
+    return config(**base)
+
+
+def test_sizes(lib):
+    c = _cfg()
+    H, Dq, Dkv, I = 2560, 4096, 1024, 9728
+    packed = lib.q3vl_packed_layer_bytes(ctypes.byref(c))
+    assert packed >= 2 * ((Dq + 2 * Dkv) * H + H * Dq + 2 * I * H + H * I)
+    S = 4096
+    ws = lib.q3vl_workspace_bytes(ctypes.byref(c), S)
+    need = 2 * S * ((Dq + 2 * Dkv) + Dq + H + I) + S * (64 * 8 + 12)
+    assert need <= ws <= need + 16 * 256
+    assert lib.q3vl_workspace_bytes(ctypes.byref(c), 0) == 0
+    assert lib.q3vl_packed_layer_bytes(ctypes.byref(_cfg(head_dim=64))) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(head_dim=64), -8), (dict(hidden=100), -1), (dict(n_heads=6, n_kv_heads=4), -1),
+    (dict(intermediate=100), -1), (dict(mrope_section=(16, 24, 24)), -8),
+])
+def test_bad_config_rejected(lib, kw, code):
+    c = _cfg(**kw)
+    rc = lib.q3vl_rope_table(ctypes.byref(c), ctypes.c_void_p(16), 8, ctypes.c_void_p(16), None)
+    assert rc == code
+    assert lib.q3vl_last_error()
+
+
+def test_empty_sequence_rejected(lib):
+    c = _cfg()
+    from qwen3_vl_decoder_b200 import _abi
+    lay = _abi.Layer(*[256] * 7)
+    rc = lib.q3vl_layer_prefill(ctypes.byref(c), ctypes.byref(lay), ctypes.c_void_p(256), 0,
+                                ctypes.c_void_p(256), None, None, 0, ctypes.c_void_p(256),
+                                1 << 40, None)
+    assert rc == -1 and b"empty" in lib.q3vl_last_error()
+
+
+def test_small_workspace_rejected(lib):
+    c = _cfg()
+    from qwen3_vl_decoder_b200 import _abi
+    lay = _abi.Layer(*[256] * 7)
+    rc = lib.q3vl_layer_prefill(ctypes.byref(c), ctypes.byref(lay), ctypes.c_void_p(256), 16,
+                                ctypes.c_void_p(256), None, None, 0, ctypes.c_void_p(256), 1024,
+                                None)
+    assert rc == -5
+
+
+def test_deepstack_contract(lib):
+    c = _cfg()
+    from qwen3_vl_decoder_b200 import _abi
+    lay = (_abi.Layer * 1)(_abi.Layer(*[256] * 7))
+    big = 1 << 40
+    slabs = (ctypes.c_void_p * 2)(256, 256)
+    # fewer than three slabs
+    rc = lib.q3vl_stack_prefill(ctypes.byref(c), 1, lay, None, ctypes.c_void_p(256), 16,
+                                ctypes.c_void_p(256), slabs, 2, ctypes.c_void_p(256), 4,
+                                ctypes.c_void_p(256), big, None)
+    assert rc == -4
+    slabs3 = (ctypes.c_void_p * 3)(256, 256, 256)
+    # slabs without image rows
+    rc = lib.q3vl_stack_prefill(ctypes.byref(c), 1, lay, None, ctypes.c_void_p(256), 16,
+                                ctypes.c_void_p(256), slabs3, 3, None, 0,
+                                ctypes.c_void_p(256), big, None)
+    assert rc == -4
+    # a layer with a slab but no rows
+    rc = lib.q3vl_layer_prefill(ctypes.byref(c), lay, ctypes.c_void_p(256), 16,
+                                ctypes.c_void_p(256), ctypes.c_void_p(256), None, 0,
+                                ctypes.c_void_p(256), big, None)
+    assert rc == -4
+
+
+def test_positions_argument_checks(lib):
+    rc = lib.q3vl_mrope_positions(ctypes.c_void_p(256), 0, None, 0, ctypes.c_void_p(256),
+                                  ctypes.c_void_p(256), None)
+    assert rc == -1
+    rc = lib.q3vl_mrope_positions(ctypes.c_void_p(256), 8, None, 1, ctypes.c_void_p(256),
+                                  ctypes.c_void_p(256), None)
+    assert rc == -1

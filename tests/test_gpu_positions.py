@@ -1,0 +1,69 @@
+"""P0 on the GPU: position ids bit-exact against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+from golden_io import all_position_files, load_positions
+from gpu_common import positions, q3
+from oracle import q3vl_oracle as O
+import q3vl_synth as syn
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(types, grids):
+    m = q3()
+    tt = torch.tensor(types, dtype=torch.uint8, device="cuda")
+    gd = torch.tensor(grids, dtype=torch.int32, device="cuda").reshape(-1, 3) if grids else None
+    return m.mrope_positions(tt, gd)
+
+
+@pytest.mark.parametrize("name", all_position_files())
+def test_golden(name):
+    types, grids, want, nxt = load_positions(name)
+    pos, got_next = _run(types, grids)
+    assert pos.cpu().tolist() == want
+    assert got_next == nxt
+
+
+@pytest.mark.parametrize("w", [syn.TINY_FP32, syn.Q2B_LAYER, syn.Q2B_STACK, syn.Q4B_LAYER,
+                               syn.Q32B_ENC, syn.Q32B_ENC_1064], ids=lambda w: w.name)
+def test_workloads(w):
+    pos, ref, nxt, ref_next = positions(w)
+    assert np.array_equal(pos.cpu().numpy(), ref)
+    assert nxt == ref_next
+
+
+def test_random_prompts_long():
+    # several chunks of the block scan, many grids, adjacent images
+    rng = np.random.default_rng(7)
+    for trial in range(20):
+        types, grids = [], []
+        while len(types) < 9000 + 500 * trial:
+            types += [0] * int(rng.integers(0, 40))
+            if rng.random() < 0.8:
+                r, c = int(rng.integers(1, 33)), int(rng.integers(1, 33))
+                types += [1] * (r * c)
+                grids.append((1, r, c))
+        pos, nxt = _run(types, grids)
+        ref, ref_next = O.mrope_positions_tokens(types, grids)
+        assert np.array_equal(pos.cpu().numpy(), ref)
+        assert nxt == ref_next
+
+
+@pytest.mark.parametrize("types,grids,code", [
+    ([0, 1, 1, 0], [(1, 1, 3)], -3),
+    ([0, 1, 1, 1], [], -3),
+    ([0, 0], [(1, 1, 1)], -3),
+    ([1, 1, 0, 1, 1], [(1, 2, 2)], -3),
+    ([1, 1], [(2, 1, 1), (1, 1, 1)], -8),
+])
+def test_mismatch_reported(types, grids, code):
+    with pytest.raises(q3().Q3VLError) as e:
+        _run(types, grids)
+    assert e.value.code == code
+
+
+def test_single_token():
+    pos, nxt = _run([0], [])
+    assert pos.cpu().tolist() == [[0], [0], [0]] and nxt == 1
