@@ -21,6 +21,14 @@ CASES = [
 ]
 
 
+def _within_output_rounding(w, got, ref):
+    """|got - ref| within the rounding of the output dtype (plus accumulation slack)."""
+    rel = 2.0 ** -8 if w.dtype == "bf16" else 2.0 ** -22
+    bound = rel * np.abs(ref) + (1e-3 if w.dtype == "bf16" else 1e-6) * np.abs(ref).mean()
+    bad = np.abs(got - ref) > bound
+    return int(bad.sum()) == 0
+
+
 def _tol(w):
     return 2e-6 if w.dtype == "fp32" else 1e-2
 
@@ -64,10 +72,13 @@ def test_steps(w):
     o_ref = O.attention(qg, kg, vg).reshape(S, -1)
     assert rel_l2(host(o), o_ref) < tol
 
-    # P6 o-projection + residual
+    # P6 o-projection + residual: exact inputs, so the only error is the
+    # output's own rounding (half an ulp of bf16 = 2^-8 relative) plus fp32
+    # accumulation order
     h = m.o_proj(cfg, packed, o, x)
     h_ref = O.o_residual(raw, host(o), xh)
-    assert rel_l2(host(h) - xh, h_ref - xh) < tol
+    assert _within_output_rounding(w, host(h), h_ref)
+    assert rel_l2(host(h) - xh, h_ref - xh) < 2 * tol
 
     # P7 + P8 post-attention norm, gate/up, SiLU * up
     inv2 = m.rms_rowstat(cfg, h)
@@ -78,7 +89,8 @@ def test_steps(w):
     # P9 down + residual
     out = m.down(cfg, packed, act, h)
     out_ref = O.down_residual(raw, host(act), host(h))
-    assert rel_l2(host(out) - host(h), out_ref - host(h)) < tol
+    assert _within_output_rounding(w, host(out), out_ref)
+    assert rel_l2(host(out) - host(h), out_ref - host(h)) < 2 * tol
     m.check_device()
 
 
@@ -100,13 +112,15 @@ def test_deepstack_down_epilogue():
     assert int((mh >= 0).sum()) == 7
     out0 = m.down(cfg, packed, act, h)
     out1 = m.down(cfg, packed, act, h, slab, dmap)
-    d = host(out1) - host(out0)
     rr = host(rows).astype(int)
-    # the slab lands on its rows (bf16 rounding of the sum), nothing elsewhere
-    assert rel_l2(d[rr], host(slab)) < 2e-2
+    # the slab lands on its rows (within the output's bf16 rounding) ...
+    ref = O.down_residual(raw, host(act), host(h))
+    ref[rr] += host(slab)
+    assert _within_output_rounding(w, host(out1), ref)
+    # ... and nowhere else (bit-identical to the call without a slab)
     mask = np.ones(w.seq, bool)
     mask[rr] = False
-    assert np.array_equal(d[mask], np.zeros_like(d[mask]))
+    assert np.array_equal(host(out1)[mask], host(out0)[mask])
     m.check_device()
 
 
