@@ -171,6 +171,24 @@ int q3vl_stack_prefill(const q3vl_config* cfg, int32_t n_layers, const q3vl_laye
                        const void* const* ds_slabs, int32_t n_ds, const int32_t* ds_rows,
                        int32_t n_img, void* ws, size_t ws_bytes, q3vl_stream stream);
 
+/* The same layer as q3vl_layer_prefill, with no workspace argument and no
+ * allocation of any kind: for callers that cannot allocate device memory (a
+ * plug-in inside a framework whose memory manager has reserved the GPU's
+ * memory, a C caller with no device allocator, a path that must not pay
+ * cudaMalloc's device-wide synchronisation). The pages have no counterpart;
+ * it exists for such callers only. Scratch is a 32 MiB array inside the
+ * library that every GPU loading it keeps until the process exits; a layer
+ * whose q3vl_workspace_bytes(cfg, S) exceeds 32 MiB is refused with
+ * Q3VL_EWORKSPACE (e.g. the 2B shape fits up to S = 1024). The first call on
+ * a device looks up the array's device address with that device current;
+ * make that first call before any stream capture. All calls share the one
+ * array: calls that overlap on the GPU (other streams, other host threads)
+ * race on it and must be serialised by the caller. Each call writes every
+ * scratch region before reading it, so nothing carries over between calls. */
+int q3vl_layer_prefill_noalloc(const q3vl_config* cfg, const q3vl_layer* layer, void* x,
+                               int64_t S, const int32_t* pos, const void* ds_slab,
+                               const int32_t* ds_rows, int32_t n_img, q3vl_stream stream);
+
 /* ---------------------------------------------------------------------------
  * Step-level calls: each step of the layer on its own, for per-step
  * parity and timing. The layer call is exactly this sequence.

@@ -153,6 +153,18 @@ def layer_prefill(cfg: Config, layer: PackedLayer, x: torch.Tensor, pos: torch.T
     return x
 
 
+def layer_prefill_noalloc(cfg: Config, layer: PackedLayer, x: torch.Tensor, pos: torch.Tensor,
+                          ds_slab: Optional[torch.Tensor] = None,
+                          ds_rows: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """layer_prefill with the library's built-in 32 MiB scratch instead of a workspace,
+    for callers that cannot allocate device memory; calls must not overlap."""
+    n_img = 0 if ds_rows is None else ds_rows.numel()
+    _check(lib().q3vl_layer_prefill_noalloc(ctypes.byref(cfg), ctypes.byref(layer.views), _ptr(x),
+                                            x.shape[0], _ptr(pos), _ptr(ds_slab), _ptr(ds_rows),
+                                            n_img, _stream(stream)))
+    return x
+
+
 def stack_prefill(cfg: Config, layers: Sequence[PackedLayer], x: torch.Tensor, pos: torch.Tensor,
                   final_norm: Optional[torch.Tensor] = None,
                   ds_slabs: Sequence[torch.Tensor] = (), ds_rows: Optional[torch.Tensor] = None,

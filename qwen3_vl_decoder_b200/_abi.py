@@ -54,6 +54,8 @@ SIGNATURES = {
     "q3vl_workspace_bytes": (_SZ, [_CFG, _I64]),
     "q3vl_layer_prefill": (ctypes.c_int, [_CFG, ctypes.POINTER(Layer), _P, _I64, _P, _P, _P, _I32,
                                           _P, _SZ, _P]),
+    "q3vl_layer_prefill_noalloc": (ctypes.c_int, [_CFG, ctypes.POINTER(Layer), _P, _I64, _P, _P,
+                                                  _P, _I32, _P]),
     "q3vl_stack_prefill": (ctypes.c_int, [_CFG, _I32, ctypes.POINTER(Layer), _P, _P, _I64, _P,
                                           ctypes.POINTER(_P), _I32, _P, _I32, _P, _SZ, _P]),
     "q3vl_rope_table": (ctypes.c_int, [_CFG, _P, _I64, _P, _P]),
