@@ -176,10 +176,10 @@ int q3vl_stack_prefill(const q3vl_config* cfg, int32_t n_layers, const q3vl_laye
  * plug-in inside a framework whose memory manager has reserved the GPU's
  * memory, a C caller with no device allocator, a path that must not pay
  * cudaMalloc's device-wide synchronisation). The pages have no counterpart;
- * it exists for such callers only. Scratch is a 32 MiB array inside the
+ * it exists for such callers only. Scratch is a 64 MiB array inside the
  * library that every GPU loading it keeps until the process exits; a layer
- * whose q3vl_workspace_bytes(cfg, S) exceeds 32 MiB is refused with
- * Q3VL_EWORKSPACE (e.g. the 2B shape fits up to S = 1024). The first call on
+ * whose q3vl_workspace_bytes(cfg, S) exceeds 64 MiB is refused with
+ * Q3VL_EWORKSPACE (e.g. the 2B shape fits up to S = 1536 on a 148-SM GPU). The first call on
  * a device looks up the array's device address with that device current;
  * make that first call before any stream capture. All calls share the one
  * array: calls that overlap on the GPU (other streams, other host threads)
@@ -192,7 +192,10 @@ int q3vl_layer_prefill_noalloc(const q3vl_config* cfg, const q3vl_layer* layer, 
 /* ---------------------------------------------------------------------------
  * Step-level calls: each step of the layer on its own, for per-step
  * parity and timing. The layer call is exactly this sequence.
- * Ntot = nh*hd + 2*nkv*hd.
+ * Ntot = nh*hd + 2*nkv*hd. The four GEMM steps (P3, P6, P8, P9) also take a
+ * layer workspace `ws` (>= q3vl_workspace_bytes(cfg, S) bytes, 256-byte
+ * aligned): only its stream-K region (fp32 partial tiles and flags for the
+ * tiles whose K range is split across CTAs) is used.
  * ------------------------------------------------------------------------- */
 
 /* P1. cos_sin[p][i] = (cos, sin)(pos[axis(i)][p] * theta^(-2i/hd)), i < hd/2,
@@ -211,7 +214,8 @@ int q3vl_rms_rowstat(const q3vl_config* cfg, const void* x, int64_t S, int64_t w
  * q,k,v = inv_rms[r] * (x W_qkv^T) + b, then each q and k head is
  * RMS-normalised with q_norm / k_norm and rotated by cos_sin. */
 int q3vl_qkv_proj(const q3vl_config* cfg, const q3vl_layer* layer, const void* x, int64_t S,
-                  const float* inv_rms, const float* cos_sin, void* qkv, q3vl_stream stream);
+                  const float* inv_rms, const float* cos_sin, void* qkv, void* ws,
+                  size_t ws_bytes, q3vl_stream stream);
 
 /* P5. o[r][h*hd + d] = causal GQA softmax attention of q head h over KV head
  * h / (nh/nkv), scale 1/sqrt(hd); qkv as written by q3vl_qkv_proj, o
@@ -221,18 +225,19 @@ int q3vl_attention(const q3vl_config* cfg, const void* qkv, int64_t S, void* o,
 
 /* P6. h = x + o Wo^T, [S, H]. */
 int q3vl_o_proj(const q3vl_config* cfg, const q3vl_layer* layer, const void* o, const void* x,
-                int64_t S, void* h, q3vl_stream stream);
+                int64_t S, void* h, void* ws, size_t ws_bytes, q3vl_stream stream);
 
 /* P8. act = silu(g) * u with [g|u] = inv_rms2[r] * (h W_gu^T), [S, I]. */
 int q3vl_gate_up(const q3vl_config* cfg, const q3vl_layer* layer, const void* h, int64_t S,
-                 const float* inv_rms2, void* act, q3vl_stream stream);
+                 const float* inv_rms2, void* act, void* ws, size_t ws_bytes,
+                 q3vl_stream stream);
 
 /* P9. out = h + act Wd^T, plus slab row ds_map[r] on rows with ds_map[r] >= 0
  * (ds_slab and ds_map may be NULL). ds_map: device int32 [S]. out may
  * equal neither h nor act. */
 int q3vl_down(const q3vl_config* cfg, const q3vl_layer* layer, const void* act, const void* h,
-              int64_t S, const void* ds_slab, const int32_t* ds_map, void* out,
-              q3vl_stream stream);
+              int64_t S, const void* ds_slab, const int32_t* ds_map, void* out, void* ws,
+              size_t ws_bytes, q3vl_stream stream);
 
 /* DeepStack row map: ds_map[r] = k if ds_rows[k] == r, else -1 (device
  * int32 [S]). Out-of-range or repeated rows record Q3VL_ERANGE. */

@@ -203,11 +203,13 @@ def _qkv_dim(cfg: Config) -> int:
     return (cfg.n_heads + 2 * cfg.n_kv_heads) * cfg.head_dim
 
 
-def qkv_proj(cfg, layer: PackedLayer, x, inv_rms, cos_sin, stream=None) -> torch.Tensor:
+def qkv_proj(cfg, layer: PackedLayer, x, inv_rms, cos_sin, ws=None, stream=None) -> torch.Tensor:
     S = x.shape[0]
+    ws = workspace(cfg, S, x.device) if ws is None else ws
     qkv = torch.empty((S, _qkv_dim(cfg)), dtype=x.dtype, device=x.device)
     _check(lib().q3vl_qkv_proj(ctypes.byref(cfg), ctypes.byref(layer.views), _ptr(x), S,
-                              _ptr(inv_rms), _ptr(cos_sin), _ptr(qkv), _stream(stream)))
+                              _ptr(inv_rms), _ptr(cos_sin), _ptr(qkv), _ptr(ws), ws.numel(),
+                              _stream(stream)))
     return qkv
 
 
@@ -218,27 +220,32 @@ def attention(cfg, qkv, stream=None) -> torch.Tensor:
     return o
 
 
-def o_proj(cfg, layer: PackedLayer, o, x, stream=None) -> torch.Tensor:
+def o_proj(cfg, layer: PackedLayer, o, x, ws=None, stream=None) -> torch.Tensor:
     S = o.shape[0]
+    ws = workspace(cfg, S, o.device) if ws is None else ws
     h = torch.empty((S, cfg.hidden), dtype=o.dtype, device=o.device)
     _check(lib().q3vl_o_proj(ctypes.byref(cfg), ctypes.byref(layer.views), _ptr(o), _ptr(x), S,
-                            _ptr(h), _stream(stream)))
+                            _ptr(h), _ptr(ws), ws.numel(), _stream(stream)))
     return h
 
 
-def gate_up(cfg, layer: PackedLayer, h, inv_rms2, stream=None) -> torch.Tensor:
+def gate_up(cfg, layer: PackedLayer, h, inv_rms2, ws=None, stream=None) -> torch.Tensor:
     S = h.shape[0]
+    ws = workspace(cfg, S, h.device) if ws is None else ws
     act = torch.empty((S, cfg.intermediate), dtype=h.dtype, device=h.device)
     _check(lib().q3vl_gate_up(ctypes.byref(cfg), ctypes.byref(layer.views), _ptr(h), S,
-                             _ptr(inv_rms2), _ptr(act), _stream(stream)))
+                             _ptr(inv_rms2), _ptr(act), _ptr(ws), ws.numel(), _stream(stream)))
     return act
 
 
-def down(cfg, layer: PackedLayer, act, h, ds_slab=None, ds_map=None, stream=None) -> torch.Tensor:
+def down(cfg, layer: PackedLayer, act, h, ds_slab=None, ds_map=None, ws=None,
+         stream=None) -> torch.Tensor:
     S = act.shape[0]
+    ws = workspace(cfg, S, act.device) if ws is None else ws
     out = torch.empty((S, cfg.hidden), dtype=act.dtype, device=act.device)
     _check(lib().q3vl_down(ctypes.byref(cfg), ctypes.byref(layer.views), _ptr(act), _ptr(h), S,
-                          _ptr(ds_slab), _ptr(ds_map), _ptr(out), _stream(stream)))
+                          _ptr(ds_slab), _ptr(ds_map), _ptr(out), _ptr(ws), ws.numel(),
+                          _stream(stream)))
     return out
 
 

@@ -60,11 +60,13 @@ SIGNATURES = {
                                           ctypes.POINTER(_P), _I32, _P, _I32, _P, _SZ, _P]),
     "q3vl_rope_table": (ctypes.c_int, [_CFG, _P, _I64, _P, _P]),
     "q3vl_rms_rowstat": (ctypes.c_int, [_CFG, _P, _I64, _I64, _P, _P]),
-    "q3vl_qkv_proj": (ctypes.c_int, [_CFG, ctypes.POINTER(Layer), _P, _I64, _P, _P, _P, _P]),
+    "q3vl_qkv_proj": (ctypes.c_int, [_CFG, ctypes.POINTER(Layer), _P, _I64, _P, _P, _P, _P, _SZ,
+                                     _P]),
     "q3vl_attention": (ctypes.c_int, [_CFG, _P, _I64, _P, _P]),
-    "q3vl_o_proj": (ctypes.c_int, [_CFG, ctypes.POINTER(Layer), _P, _P, _I64, _P, _P]),
-    "q3vl_gate_up": (ctypes.c_int, [_CFG, ctypes.POINTER(Layer), _P, _I64, _P, _P, _P]),
-    "q3vl_down": (ctypes.c_int, [_CFG, ctypes.POINTER(Layer), _P, _P, _I64, _P, _P, _P, _P]),
+    "q3vl_o_proj": (ctypes.c_int, [_CFG, ctypes.POINTER(Layer), _P, _P, _I64, _P, _P, _SZ, _P]),
+    "q3vl_gate_up": (ctypes.c_int, [_CFG, ctypes.POINTER(Layer), _P, _I64, _P, _P, _P, _SZ, _P]),
+    "q3vl_down": (ctypes.c_int, [_CFG, ctypes.POINTER(Layer), _P, _P, _I64, _P, _P, _P, _P, _SZ,
+                                 _P]),
     "q3vl_deepstack_map": (ctypes.c_int, [_P, _I32, _I64, _P, _P]),
     "q3vl_final_norm": (ctypes.c_int, [_CFG, _P, _I64, _P, _P]),
     "q3vl_device_status": (ctypes.c_int, [_P, ctypes.POINTER(_I32), ctypes.POINTER(_I32)]),

@@ -67,6 +67,11 @@ WsLayout ws_layout(const q3vl_config& c, int64_t S) {
   L.o = take(size_t(S) * q_dim(c) * e);
   L.h = take(size_t(S) * c.hidden * e);
   L.act = take(size_t(S) * c.intermediate * e);
+  if (c.dtype == Q3VL_DTYPE_BF16) {
+    L.sk_slots = sm_count();
+    L.sk_part = take(size_t(L.sk_slots) * kSkSlotBytes);
+    L.sk_flags = take(size_t(L.sk_slots) * sizeof(int32_t));
+  }
   L.total = off;
   return L;
 }
@@ -202,13 +207,44 @@ namespace {
 
 bool is_bf16(const q3vl_config& c) { return c.dtype == Q3VL_DTYPE_BF16; }
 
+// Stream-K scratch of a layer workspace.
+struct Sk {
+  float* part = nullptr;
+  int32_t* flags = nullptr;
+  int slots = 0;
+};
+
+Sk sk_of(const WsLayout& L, char* ws) {
+  Sk k;
+  if (L.sk_slots > 0) {
+    k.part = reinterpret_cast<float*>(ws + L.sk_part);
+    k.flags = reinterpret_cast<int32_t*>(ws + L.sk_flags);
+    k.slots = L.sk_slots;
+  }
+  return k;
+}
+
+void set_sk(GemmArgs& a, const Sk& k) {
+  a.sk_partials = k.part;
+  a.sk_flags = k.flags;
+  a.sk_slots = k.slots;
+  a.sk_slot_bytes = kSkSlotBytes;
+}
+
+int clear_sk_flags(const Sk& k, cudaStream_t st) {
+  if (k.flags == nullptr) return Q3VL_OK;
+  return cuda_check(cudaMemsetAsync(k.flags, 0, size_t(k.slots) * sizeof(int32_t), st),
+                    "clear stream-K flags");
+}
+
 int run_qkv(const q3vl_config& c, const q3vl_layer& w, const void* x, int64_t S, const float* inv,
-            const float* cs, void* qkv, cudaStream_t st) {
+            const float* cs, void* qkv, const Sk& sk, cudaStream_t st) {
   GemmArgs a{};
   a.A = x; a.B = w.w_qkv; a.M = S; a.N = qkv_dim(c); a.K = c.hidden;
   a.out = qkv; a.ldo = a.N; a.row_scale = inv; a.bias = w.b_qkv;
   a.q_norm = w.q_norm; a.k_norm = w.k_norm; a.cos_sin = cs;
   a.q_cols = q_dim(c); a.k_cols = kv_dim(c); a.eps = static_cast<float>(c.rms_eps);
+  set_sk(a, sk);
   if (is_bf16(c)) return cuda_check(launch_gemm_tc(Epi::kQkv, a, st), "qkv projection");
   Q3VL_CUDA(launch_gemm_f32(Epi::kPlain, a, st), "qkv projection");
   return cuda_check(launch_qk_norm_rope_f32(c, static_cast<float*>(qkv), S, w.q_norm, w.k_norm,
@@ -224,20 +260,22 @@ int run_attention(const q3vl_config& c, const void* qkv, int64_t S, void* o, cud
 }
 
 int run_oproj(const q3vl_config& c, const q3vl_layer& w, const void* o, const void* x, int64_t S,
-              void* h, cudaStream_t st) {
+              void* h, const Sk& sk, cudaStream_t st) {
   GemmArgs a{};
   a.A = o; a.B = w.w_o; a.M = S; a.N = c.hidden; a.K = q_dim(c);
   a.out = h; a.ldo = c.hidden; a.resid = x;
+  set_sk(a, sk);
   if (is_bf16(c)) return cuda_check(launch_gemm_tc(Epi::kResidual, a, st), "o projection");
   return cuda_check(launch_gemm_f32(Epi::kResidual, a, st), "o projection");
 }
 
 int run_gateup(const q3vl_config& c, const q3vl_layer& w, const void* h, int64_t S,
-               const float* inv2, void* act, cudaStream_t st) {
+               const float* inv2, void* act, const Sk& sk, cudaStream_t st) {
   if (is_bf16(c)) {
     GemmArgs a{};
     a.A = h; a.B = w.w_gu; a.M = S; a.N = 2 * int64_t(c.intermediate); a.K = c.hidden;
     a.out = act; a.ldo = c.intermediate; a.row_scale = inv2;
+    set_sk(a, sk);
     return cuda_check(launch_gemm_tc(Epi::kSwiGLU, a, st), "gate/up projection");
   }
   return cuda_check(launch_gemm_swiglu_f32(static_cast<const float*>(h),
@@ -247,12 +285,13 @@ int run_gateup(const q3vl_config& c, const q3vl_layer& w, const void* h, int64_t
 }
 
 int run_down(const q3vl_config& c, const q3vl_layer& w, const void* act, const void* h, int64_t S,
-             const void* ds_slab, const int32_t* ds_map, void* out, cudaStream_t st) {
+             const void* ds_slab, const int32_t* ds_map, void* out, const Sk& sk, cudaStream_t st) {
   GemmArgs a{};
   a.A = act; a.B = w.w_down; a.M = S; a.N = c.hidden; a.K = c.intermediate;
   a.out = out; a.ldo = c.hidden; a.resid = h;
   a.ds_slab = ds_map ? ds_slab : nullptr;
   a.ds_map = ds_slab ? ds_map : nullptr;
+  set_sk(a, sk);
   if (is_bf16(c)) return cuda_check(launch_gemm_tc(Epi::kResidual, a, st), "down projection");
   return cuda_check(launch_gemm_f32(Epi::kResidual, a, st), "down projection");
 }
@@ -269,19 +308,20 @@ int run_layer(const q3vl_config& c, const q3vl_layer& w, void* x, int64_t S, cha
   void* o = ws + L.o;
   void* h = ws + L.h;
   void* act = ws + L.act;
+  const Sk sk = sk_of(L, ws);
   Q3VL_CUDA(launch_rowstat(c, x, S, c.hidden, inv1, st), "input rms");
   stage_event(2, st);
-  Q3VL_TRY(run_qkv(c, w, x, S, inv1, cs, qkv, st));
+  Q3VL_TRY(run_qkv(c, w, x, S, inv1, cs, qkv, sk, st));
   stage_event(3, st);
   Q3VL_TRY(run_attention(c, qkv, S, o, st));
   stage_event(4, st);
-  Q3VL_TRY(run_oproj(c, w, o, x, S, h, st));
+  Q3VL_TRY(run_oproj(c, w, o, x, S, h, sk, st));
   stage_event(5, st);
   Q3VL_CUDA(launch_rowstat(c, h, S, c.hidden, inv2, st), "post-attention rms");
   stage_event(6, st);
-  Q3VL_TRY(run_gateup(c, w, h, S, inv2, act, st));
+  Q3VL_TRY(run_gateup(c, w, h, S, inv2, act, sk, st));
   stage_event(7, st);
-  Q3VL_TRY(run_down(c, w, act, h, S, ds_slab, ds_slab ? map : nullptr, x, st));
+  Q3VL_TRY(run_down(c, w, act, h, S, ds_slab, ds_slab ? map : nullptr, x, sk, st));
   stage_event(8, st);
   return Q3VL_OK;
 }
@@ -301,6 +341,14 @@ int check_ptr(const void* p, const char* name, bool need16 = true) {
   if (need16 && (reinterpret_cast<uintptr_t>(p) & 15) != 0)
     return set_error(Q3VL_EINVAL, std::string(name) + " must be 16-byte aligned");
   return Q3VL_OK;
+}
+
+// Stream-K scratch of a step-level GEMM call: the workspace's stream-K
+// region, flags cleared on the stream first.
+int step_sk(const q3vl_config& c, int64_t S, void* ws, size_t ws_bytes, cudaStream_t st, Sk* out) {
+  Q3VL_TRY(check_ws(c, S, ws, ws_bytes));
+  *out = sk_of(ws_layout(c, S), static_cast<char*>(ws));
+  return clear_sk_flags(*out, st);
 }
 
 }  // namespace
@@ -388,7 +436,8 @@ int q3vl_rms_rowstat(const q3vl_config* cfg, const void* x, int64_t S, int64_t w
 }
 
 int q3vl_qkv_proj(const q3vl_config* cfg, const q3vl_layer* layer, const void* x, int64_t S,
-                  const float* inv_rms, const float* cos_sin, void* qkv, q3vl_stream stream) {
+                  const float* inv_rms, const float* cos_sin, void* qkv, void* ws,
+                  size_t ws_bytes, q3vl_stream stream) {
   Q3VL_TRY(check_cfg(cfg));
   Q3VL_TRY(check_seq(S));
   Q3VL_TRY(check_layer(cfg, layer));
@@ -396,7 +445,9 @@ int q3vl_qkv_proj(const q3vl_config* cfg, const q3vl_layer* layer, const void* x
   Q3VL_TRY(check_ptr(inv_rms, "inv_rms", false));
   Q3VL_TRY(check_ptr(cos_sin, "cos_sin"));
   Q3VL_TRY(check_ptr(qkv, "qkv"));
-  return run_qkv(*cfg, *layer, x, S, inv_rms, cos_sin, qkv, ST(stream));
+  Sk sk;
+  Q3VL_TRY(step_sk(*cfg, S, ws, ws_bytes, ST(stream), &sk));
+  return run_qkv(*cfg, *layer, x, S, inv_rms, cos_sin, qkv, sk, ST(stream));
 }
 
 int q3vl_attention(const q3vl_config* cfg, const void* qkv, int64_t S, void* o,
@@ -409,30 +460,35 @@ int q3vl_attention(const q3vl_config* cfg, const void* qkv, int64_t S, void* o,
 }
 
 int q3vl_o_proj(const q3vl_config* cfg, const q3vl_layer* layer, const void* o, const void* x,
-                int64_t S, void* h, q3vl_stream stream) {
+                int64_t S, void* h, void* ws, size_t ws_bytes, q3vl_stream stream) {
   Q3VL_TRY(check_cfg(cfg));
   Q3VL_TRY(check_seq(S));
   Q3VL_TRY(check_layer(cfg, layer));
   Q3VL_TRY(check_ptr(o, "o"));
   Q3VL_TRY(check_ptr(x, "x"));
   Q3VL_TRY(check_ptr(h, "h"));
-  return run_oproj(*cfg, *layer, o, x, S, h, ST(stream));
+  Sk sk;
+  Q3VL_TRY(step_sk(*cfg, S, ws, ws_bytes, ST(stream), &sk));
+  return run_oproj(*cfg, *layer, o, x, S, h, sk, ST(stream));
 }
 
 int q3vl_gate_up(const q3vl_config* cfg, const q3vl_layer* layer, const void* h, int64_t S,
-                 const float* inv_rms2, void* act, q3vl_stream stream) {
+                 const float* inv_rms2, void* act, void* ws, size_t ws_bytes,
+                 q3vl_stream stream) {
   Q3VL_TRY(check_cfg(cfg));
   Q3VL_TRY(check_seq(S));
   Q3VL_TRY(check_layer(cfg, layer));
   Q3VL_TRY(check_ptr(h, "h"));
   Q3VL_TRY(check_ptr(inv_rms2, "inv_rms2", false));
   Q3VL_TRY(check_ptr(act, "act"));
-  return run_gateup(*cfg, *layer, h, S, inv_rms2, act, ST(stream));
+  Sk sk;
+  Q3VL_TRY(step_sk(*cfg, S, ws, ws_bytes, ST(stream), &sk));
+  return run_gateup(*cfg, *layer, h, S, inv_rms2, act, sk, ST(stream));
 }
 
 int q3vl_down(const q3vl_config* cfg, const q3vl_layer* layer, const void* act, const void* h,
-              int64_t S, const void* ds_slab, const int32_t* ds_map, void* out,
-              q3vl_stream stream) {
+              int64_t S, const void* ds_slab, const int32_t* ds_map, void* out, void* ws,
+              size_t ws_bytes, q3vl_stream stream) {
   Q3VL_TRY(check_cfg(cfg));
   Q3VL_TRY(check_seq(S));
   Q3VL_TRY(check_layer(cfg, layer));
@@ -443,7 +499,9 @@ int q3vl_down(const q3vl_config* cfg, const q3vl_layer* layer, const void* act, 
     return set_error(Q3VL_EDEEPSTACK, "ds_slab and ds_map must both be given or both be NULL");
   if (ds_slab) Q3VL_TRY(check_ptr(ds_slab, "ds_slab"));
   if (out == h || out == act) return set_error(Q3VL_EINVAL, "out must not alias h or act");
-  return run_down(*cfg, *layer, act, h, S, ds_slab, ds_map, out, ST(stream));
+  Sk sk;
+  Q3VL_TRY(step_sk(*cfg, S, ws, ws_bytes, ST(stream), &sk));
+  return run_down(*cfg, *layer, act, h, S, ds_slab, ds_map, out, sk, ST(stream));
 }
 
 int q3vl_deepstack_map(const int32_t* ds_rows, int32_t n_img, int64_t S, int32_t* ds_map,
@@ -483,6 +541,7 @@ int q3vl_layer_prefill(const q3vl_config* cfg, const q3vl_layer* layer, void* x,
   const WsLayout L = ws_layout(*cfg, S);
   char* w = static_cast<char*>(ws);
   stage_event(0, st);
+  Q3VL_TRY(clear_sk_flags(sk_of(L, w), st));
   Q3VL_CUDA(launch_rope_table(*cfg, pos, S, reinterpret_cast<float*>(w + L.cos_sin), st),
             "rope table");
   if (ds_slab != nullptr)
@@ -522,6 +581,7 @@ int q3vl_stack_prefill(const q3vl_config* cfg, int32_t n_layers, const q3vl_laye
   const cudaStream_t st = ST(stream);
   const WsLayout L = ws_layout(*cfg, S);
   char* w = static_cast<char*>(ws);
+  Q3VL_TRY(clear_sk_flags(sk_of(L, w), st));
   Q3VL_CUDA(launch_rope_table(*cfg, pos, S, reinterpret_cast<float*>(w + L.cos_sin), st),
             "rope table");
   if (n_ds > 0)

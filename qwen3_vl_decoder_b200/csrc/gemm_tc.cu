@@ -58,7 +58,96 @@ struct Params {
   const __nv_bfloat16* ds_slab;
   const int32_t* ds_map;
   int32_t* err;
+  // schedule (see Sched)
+  int64_t dp_tiles, sk_units;
+  int kb_per_tile;
+  // stream-K scratch: one fp32 partial tile per CTA and one flag per CTA
+  float* sk_partials;
+  int32_t* sk_flags;
 };
+
+// Work schedule shared by the three roles of a CTA.
+//   tiles [0, dp_tiles): data parallel; CTA c takes tiles c, c + G, ... over
+//     their whole K range;
+//   tiles [dp_tiles, T): stream-K; their U = (T - dp_tiles) * KB k-block
+//     units are cut into G equal contiguous ranges, CTA c taking units
+//     [c U / G, (c + 1) U / G).
+// A stream-K tile split across CTAs is finished by the CTA holding its first
+// k-block, which reaches it last in time (at the end of its range). The CTAs
+// holding its later k-blocks reach them first (at the start of their
+// ranges): they leave fp32 partial sums in their own scratch slot and raise
+// their flag; the finisher adds the partials in CTA order (deterministic)
+// before the fused epilogue.
+enum Role : int { kFull = 0, kFinisher = 1, kContributor = 2 };
+
+struct Work {
+  int64_t tile;
+  int kb0, kb1, role;
+};
+
+struct WorkIter {
+  int64_t dp_t, dp_tiles, stride;  // data-parallel part
+  int64_t u, u1, sk_base;          // stream-K part (units relative to tile dp_tiles)
+  int KB;
+  __device__ WorkIter(const Params& p, int c, int G)
+      : dp_t(c), dp_tiles(p.dp_tiles), stride(G), u(p.sk_units * c / G),
+        u1(p.sk_units * (c + 1) / G), sk_base(p.dp_tiles), KB(p.kb_per_tile) {}
+  __device__ bool next(Work& w) {
+    if (dp_t < dp_tiles) {
+      w.tile = dp_t; w.kb0 = 0; w.kb1 = KB; w.role = kFull;
+      dp_t += stride;
+      return true;
+    }
+    if (u >= u1) return false;
+    const int64_t t = u / KB;
+    const int64_t end = min(u1, (t + 1) * KB);
+    w.tile = sk_base + t;
+    w.kb0 = static_cast<int>(u - t * KB);
+    w.kb1 = static_cast<int>(end - t * KB);
+    w.role = w.kb0 > 0 ? kContributor : (w.kb1 == KB ? kFull : kFinisher);
+    u = end;
+    return true;
+  }
+};
+
+// Owner CTA of stream-K unit u: the largest c with c U / G <= u.
+__device__ __forceinline__ int sk_owner(int64_t u, int64_t U, int G) {
+  return static_cast<int>(((u + 1) * G - 1) / U);
+}
+
+__device__ __forceinline__ int ld_acquire(const int32_t* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release(int32_t* p, int v) {
+  asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Named barrier over the four epilogue warps only.
+__device__ __forceinline__ void epilogue_sync() { asm volatile("barrier.sync 1, 128;" ::: "memory"); }
+
+// Loads accumulator columns [32 cc, 32 cc + 32) of this thread's row from
+// TMEM and adds the partial sums of n_part contributor slots (fp32).
+template <int BN>
+__device__ __forceinline__ void load_chunk(uint32_t taddr, int cc, int rr, const float* part,
+                                           int n_part, float* v) {
+  uint32_t r[32];
+  tmem_ld32(taddr, r);
+  tmem_ld_wait();
+#pragma unroll
+  for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(r[t]);
+  for (int i = 0; i < n_part; ++i) {
+    const float4* src = reinterpret_cast<const float4*>(
+        part + static_cast<size_t>(i) * (BM * BN) + (static_cast<size_t>(cc) * BM + rr) * 32);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float4 q = __ldcg(src + j);
+      v[4 * j] += q.x; v[4 * j + 1] += q.y; v[4 * j + 2] += q.z; v[4 * j + 3] += q.w;
+    }
+  }
+}
 
 __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float* v) {
   uint4* d = reinterpret_cast<uint4*>(dst);
@@ -85,19 +174,17 @@ __device__ __forceinline__ void add_bf16x32(float* v, const __nv_bfloat16* src) 
 }
 
 // One 128-column head of the QKV epilogue for this thread's row.
-__device__ __forceinline__ void qkv_head(uint32_t taddr, int64_t row, bool valid, int64_t c0,
+template <int BN>
+__device__ __forceinline__ void qkv_head(uint32_t taddr, int cc0, int rr, const float* part,
+                                         int n_part, int64_t row, bool valid, int64_t c0,
                                          const Params& p) {
-  uint32_t raw[4][32];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) tmem_ld32(taddr + 32 * j, raw[j]);
-  tmem_ld_wait();
-  if (!valid) return;
   float v[128];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) load_chunk<BN>(taddr + 32 * j, cc0 + j, rr, part, n_part, v + 32 * j);
+  if (!valid) return;
   const float s = p.row_scale[row];
 #pragma unroll
-  for (int j = 0; j < 4; ++j)
-#pragma unroll
-    for (int t = 0; t < 32; ++t) v[32 * j + t] = __uint_as_float(raw[j][t]) * s;
+  for (int t = 0; t < 128; ++t) v[t] *= s;
   if (p.bias != nullptr) {
     const float4* b = reinterpret_cast<const float4*>(p.bias + c0);
 #pragma unroll
@@ -175,20 +262,21 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const uint32_t tmem_base = *tmem_slot;
 
   const int64_t num_m = (p.M + BM - 1) / BM;
-  const int64_t num_n = p.N / BN;
-  const int64_t total = num_m * num_n;
-  const int nk = static_cast<int>(p.K / BK);
+  const int G = static_cast<int>(gridDim.x);
+  const int c = static_cast<int>(blockIdx.x);
 
   if (warp == 0) {
     if (lane == 0) {
       int stage = 0;
       uint32_t ph = 0;
       uint32_t issued = 0, last_ph = 0;  // per-stage bit masks
-      for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x) {
-        const int32_t m0 = static_cast<int32_t>((tile % num_m) * BM);
-        const int32_t n0 = static_cast<int32_t>((tile / num_m) * BN);
-        bool ok = true;
-        for (int kb = 0; kb < nk; ++kb) {
+      WorkIter it(p, c, G);
+      Work w;
+      bool ok = true;
+      while (ok && it.next(w)) {
+        const int32_t m0 = static_cast<int32_t>((w.tile % num_m) * BM);
+        const int32_t n0 = static_cast<int32_t>((w.tile / num_m) * BN);
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
           if (!mbar_wait(empty + stage, ph ^ 1, p.err, kWhereGemmProducer, abort_flag)) {
             ok = false;
             break;
@@ -200,7 +288,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           last_ph = (last_ph & ~(1u << stage)) | (ph << stage);
           if (++stage == S) { stage = 0; ph ^= 1; }
         }
-        if (!ok) break;
       }
       // Every issued load must land before the block exits.
       for (int s = 0; s < S; ++s)
@@ -213,14 +300,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       int stage = 0;
       uint32_t ph = 0;
       int acc_i = 0;
-      for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x, ++acc_i) {
+      WorkIter it(p, c, G);
+      Work w;
+      bool ok = true;
+      while (ok && it.next(w)) {
         const int buf = acc_i & 1;
         if (!mbar_wait(tempty + buf, ((acc_i >> 1) & 1) ^ 1, p.err, kWhereGemmMma, abort_flag))
           break;
         tc_fence_after();
         const uint32_t d = tmem_base + buf * BN;
-        bool ok = true;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
           if (!mbar_wait(full + stage, ph, p.err, kWhereGemmMma, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_u32(smA + stage * C::kABytes);
@@ -228,12 +317,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
             umma_bf16_ss(d, sdesc_sw128(a0 + 32 * k, 16, 1024), sdesc_sw128(b0 + 32 * k, 16, 1024),
-                         idesc, (kb | k) != 0);
+                         idesc, (kb > w.kb0 || k > 0) ? 1u : 0u);
           umma_commit(empty + stage);
           if (++stage == S) { stage = 0; ph ^= 1; }
         }
         if (!ok) break;
         umma_commit(tfull + buf);
+        ++acc_i;
       }
       // All issued MMAs complete before TMEM is released.
       umma_commit(drain);
@@ -242,59 +332,102 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   } else {
     const int quarter = warp & 3;
     const int rr = quarter * 32 + lane;
+    const bool leader = warp == 2 && lane == 0;
     const uint32_t lane_field = static_cast<uint32_t>(quarter * 32) << 16;
     int acc_i = 0;
-    for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x, ++acc_i) {
+    WorkIter it(p, c, G);
+    Work w;
+    while (it.next(w)) {
       const int buf = acc_i & 1;
       bool ok = mbar_wait(tfull + buf, (acc_i >> 1) & 1, p.err, kWhereGemmEpilogue, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      const int64_t row = (tile % num_m) * BM + rr;
-      const int64_t n0 = (tile / num_m) * BN;
+      const int64_t row = (w.tile % num_m) * BM + rr;
+      const int64_t n0 = (w.tile / num_m) * BN;
       const bool valid = row < p.M;
       const uint32_t tbase = tmem_base + buf * BN + lane_field;
-      if constexpr (EPI == static_cast<int>(Epi::kQkv)) {
-#pragma unroll 1
-        for (int hh = 0; hh < BN / 128; ++hh) qkv_head(tbase + 128 * hh, row, valid, n0 + 128 * hh, p);
-      } else if constexpr (EPI == static_cast<int>(Epi::kSwiGLU)) {
-        const float s = valid ? p.row_scale[row] : 0.f;
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t g[32], u[32];
-          tmem_ld32(tbase + 32 * cc, g);
-          tmem_ld32(tbase + 128 + 32 * cc, u);
-          tmem_ld_wait();
-          if (valid) {
-            float v[32];
-#pragma unroll
-            for (int t = 0; t < 32; ++t)
-              v[t] = silu_f(__uint_as_float(g[t]) * s) * (__uint_as_float(u[t]) * s);
-            store_bf16x32(p.out + row * p.ldo + n0 / 2 + 32 * cc, v);
-          }
-        }
-      } else {
-        const int32_t dsk = (EPI == static_cast<int>(Epi::kResidual) && valid && p.ds_map != nullptr)
-                                ? p.ds_map[row] : -1;
+      if (w.role == kContributor) {
+        // leave the fp32 partial tile in this CTA's slot, then raise the flag
+        float* slot = p.sk_partials + static_cast<size_t>(c) * (BM * BN);
 #pragma unroll 1
         for (int cc = 0; cc < BN / 32; ++cc) {
-          uint32_t a[32];
-          tmem_ld32(tbase + 32 * cc, a);
+          uint32_t r[32];
+          tmem_ld32(tbase + 32 * cc, r);
           tmem_ld_wait();
-          if (valid) {
-            float v[32];
+          float4* dst = reinterpret_cast<float4*>(slot + (static_cast<size_t>(cc) * BM + rr) * 32);
 #pragma unroll
-            for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(a[t]);
-            const int64_t col = n0 + 32 * cc;
-            if constexpr (EPI == static_cast<int>(Epi::kResidual)) {
-              add_bf16x32(v, p.resid + row * p.ldo + col);
-              if (dsk >= 0) add_bf16x32(v, p.ds_slab + int64_t(dsk) * p.N + col);
+          for (int j = 0; j < 8; ++j)
+            __stcg(dst + j, make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                        __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])));
+        }
+        __threadfence();
+        epilogue_sync();
+        if (leader) st_release(p.sk_flags + c, 1);
+      } else {
+        const float* part = nullptr;
+        int n_part = 0;
+        if (w.role == kFinisher) {
+          // contributors: the CTAs owning k-blocks [kb1, KB) of this tile
+          const int64_t t_rel = w.tile - p.dp_tiles;
+          const int c_last = sk_owner((t_rel + 1) * p.kb_per_tile - 1, p.sk_units, G);
+          part = p.sk_partials + static_cast<size_t>(c + 1) * (BM * BN);
+          n_part = c_last - c;
+          if (leader) {
+            for (int cp = c + 1; cp <= c_last; ++cp) {
+              const uint64_t t0 = globaltimer_ns();
+              while (ld_acquire(p.sk_flags + cp) != 1) {
+                if (*abort_flag) break;
+                if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                  record_error(p.err, Q3VL_ETIMEOUT, kWhereGemmEpilogue);
+                  *abort_flag = 1;
+                  break;
+                }
+              }
+              p.sk_flags[cp] = 0;  // ready for the next launch on this workspace
             }
-            store_bf16x32(p.out + row * p.ldo + col, v);
+          }
+          epilogue_sync();
+        }
+        if constexpr (EPI == static_cast<int>(Epi::kQkv)) {
+#pragma unroll 1
+          for (int hh = 0; hh < BN / 128; ++hh)
+            qkv_head<BN>(tbase + 128 * hh, 4 * hh, rr, part, n_part, row, valid, n0 + 128 * hh, p);
+        } else if constexpr (EPI == static_cast<int>(Epi::kSwiGLU)) {
+          const float s = valid ? p.row_scale[row] : 0.f;
+#pragma unroll 1
+          for (int cc = 0; cc < 4; ++cc) {
+            float g[32], u[32];
+            load_chunk<BN>(tbase + 32 * cc, cc, rr, part, n_part, g);
+            load_chunk<BN>(tbase + 128 + 32 * cc, cc + 4, rr, part, n_part, u);
+            if (valid) {
+              float v[32];
+#pragma unroll
+              for (int t = 0; t < 32; ++t) v[t] = silu_f(g[t] * s) * (u[t] * s);
+              store_bf16x32(p.out + row * p.ldo + n0 / 2 + 32 * cc, v);
+            }
+          }
+        } else {
+          const int32_t dsk =
+              (EPI == static_cast<int>(Epi::kResidual) && valid && p.ds_map != nullptr)
+                  ? p.ds_map[row] : -1;
+#pragma unroll 1
+          for (int cc = 0; cc < BN / 32; ++cc) {
+            float v[32];
+            load_chunk<BN>(tbase + 32 * cc, cc, rr, part, n_part, v);
+            if (valid) {
+              const int64_t col = n0 + 32 * cc;
+              if constexpr (EPI == static_cast<int>(Epi::kResidual)) {
+                add_bf16x32(v, p.resid + row * p.ldo + col);
+                if (dsk >= 0) add_bf16x32(v, p.ds_slab + int64_t(dsk) * p.N + col);
+              }
+              store_bf16x32(p.out + row * p.ldo + col, v);
+            }
           }
         }
       }
       tc_fence_before();
       mbar_arrive(tempty + buf);
+      ++acc_i;
     }
   }
   tc_fence_before();
@@ -305,8 +438,39 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   }
 }
 
+// Host-side schedule: data-parallel waves, and stream-K over the remainder
+// when the last wave would leave many SMs idle.
+struct HostSched {
+  int grid;
+  int64_t dp_tiles, sk_units;
+};
+
+HostSched make_sched(int64_t tiles, int kb, int sms) {
+  HostSched h{};
+  const int64_t rem = tiles % sms;
+  if (rem == 0 || (tiles >= sms && rem * 100 >= 92LL * sms)) {
+    h.grid = static_cast<int>(tiles < sms ? tiles : sms);
+    h.dp_tiles = tiles;
+    h.sk_units = 0;
+    return h;
+  }
+  const int64_t waves = tiles / sms;
+  h.dp_tiles = waves > 0 ? (waves - 1) * sms : 0;
+  h.sk_units = (tiles - h.dp_tiles) * kb;
+  int64_t g = sms;
+  if (tiles < sms) {
+    // small problems: whole tiles, or at least 8 k-blocks per CTA
+    const int64_t by_units = (h.sk_units + 7) / 8;
+    g = tiles > by_units ? tiles : by_units;
+    if (g > sms) g = sms;
+  }
+  if (g > h.sk_units) g = h.sk_units;
+  h.grid = static_cast<int>(g);
+  return h;
+}
+
 template <int BN, int EPI>
-cudaError_t launch_bn(const GemmArgs& a, const Params& p, cudaStream_t st) {
+cudaError_t launch_bn(const GemmArgs& a, Params p, cudaStream_t st) {
   using C = Cfg<BN>;
   CUtensorMap tmA, tmB;
   if (!make_tmap_bf16(&tmA, a.A, a.M, a.K, a.K, BK, BM)) return cudaErrorInvalidValue;
@@ -316,21 +480,22 @@ cudaError_t launch_bn(const GemmArgs& a, const Params& p, cudaStream_t st) {
                                        static_cast<int>(C::kSmem));
   if (e != cudaSuccess) return e;
   const int64_t tiles = ((a.M + BM - 1) / BM) * (a.N / BN);
-  const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
-  kern<<<grid, kThreads, C::kSmem, st>>>(tmA, tmB, p);
+  const HostSched h = make_sched(tiles, static_cast<int>(a.K / BK), sm_count());
+  if (h.sk_units > 0 &&
+      (a.sk_partials == nullptr || a.sk_flags == nullptr || h.grid > a.sk_slots ||
+       size_t(BM) * BN * sizeof(float) > a.sk_slot_bytes))
+    return cudaErrorInvalidValue;
+  p.dp_tiles = h.dp_tiles;
+  p.sk_units = h.sk_units;
+  p.kb_per_tile = static_cast<int>(a.K / BK);
+  kern<<<h.grid, kThreads, C::kSmem, st>>>(tmA, tmB, p);
   return counted_launch(1);
-}
-
-// Fraction of SM-slots doing work over all waves of a persistent grid.
-double wave_efficiency(int64_t tiles, int sms) {
-  const int64_t waves = (tiles + sms - 1) / sms;
-  return static_cast<double>(tiles) / static_cast<double>(waves * sms);
 }
 
 }  // namespace
 
 cudaError_t launch_gemm_tc(Epi epi, const GemmArgs& a, cudaStream_t st) {
-  Params p;
+  Params p{};
   p.M = a.M; p.N = a.N; p.K = a.K;
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.ldo = a.ldo;
@@ -341,12 +506,12 @@ cudaError_t launch_gemm_tc(Epi epi, const GemmArgs& a, cudaStream_t st) {
   p.ds_slab = static_cast<const __nv_bfloat16*>(a.ds_slab);
   p.ds_map = a.ds_map;
   p.err = device_error_ptr();
+  p.sk_partials = a.sk_partials;
+  p.sk_flags = a.sk_flags;
   if (a.K % BK != 0 || a.N % 128 != 0 || a.M <= 0) return cudaErrorInvalidValue;
-  const int sms = sm_count();
-  const int64_t mt = (a.M + BM - 1) / BM;
-  bool use256 = a.N % 256 == 0;
-  if (use256 && epi != Epi::kSwiGLU)
-    use256 = wave_efficiency(mt * (a.N / 256), sms) >= wave_efficiency(mt * (a.N / 128), sms) - 1e-9;
+  // 128 x 256 tiles: a 128-wide N tile makes a single-CTA tcgen05.mma
+  // shared-memory-bandwidth bound; stream-K absorbs the wave quantization.
+  const bool use256 = a.N % 256 == 0;
   switch (epi) {
     case Epi::kQkv:
       return use256 ? launch_bn<256, 0>(a, p, st) : launch_bn<128, 0>(a, p, st);

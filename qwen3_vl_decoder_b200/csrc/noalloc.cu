@@ -9,7 +9,7 @@
 // positions and the packed weights; only the scratch space is built in.
 //
 // The scratch is one file-scope device array of kNoAllocScratchBytes
-// (32 MiB). Every GPU that loads this library keeps that array for the life
+// (64 MiB). Every GPU that loads this library keeps that array for the life
 // of the process. Its device address is looked up once per device, on the
 // first call made with that device current (cudaGetSymbolAddress), so make
 // that first call before any stream capture. All calls share the one array:
@@ -26,7 +26,7 @@
 namespace q3vl {
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 

@@ -15,6 +15,7 @@ namespace q3vl {
 
 constexpr int kHeadDim = 128;
 constexpr int kHalf = kHeadDim / 2;
+constexpr size_t kSkSlotBytes = size_t(128) * 256 * sizeof(float);
 
 inline size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
@@ -33,6 +34,9 @@ struct WsLayout {
   size_t o = 0;        // dtype [S][Dq]
   size_t h = 0;        // dtype [S][H]
   size_t act = 0;      // dtype [S][I]
+  size_t sk_part = 0;  // fp32 [sk_slots][128 x 256] stream-K partial tiles
+  size_t sk_flags = 0; // int32 [sk_slots], zero between GEMM launches
+  int sk_slots = 0;
   size_t total = 0;
 };
 WsLayout ws_layout(const q3vl_config& c, int64_t S);
@@ -90,6 +94,12 @@ struct GemmArgs {
   const void* resid;       // bf16 [M, ldo] (kResidual)
   const void* ds_slab;     // bf16 [n_img, N] (kResidual) or null
   const int32_t* ds_map;   // [M] (kResidual) or null
+  // stream-K scratch (bf16 tensor-core path): sk_slots fp32 partial tiles
+  // of sk_slot_bytes each, and sk_slots int32 flags that start at zero
+  float* sk_partials;
+  int32_t* sk_flags;
+  int sk_slots;
+  size_t sk_slot_bytes;
 };
 cudaError_t launch_gemm_tc(Epi epi, const GemmArgs& a, cudaStream_t st);
 cudaError_t launch_attention_tc(const q3vl_config& c, const void* qkv, int64_t S, void* o,

@@ -62,7 +62,7 @@ def test_noalloc_matches_workspace_entry_point_twice(w):
 
 def test_noalloc_refuses_layers_above_its_scratch():
     m = q3()
-    w = syn.Q2B_LAYER.with_seq(1200)   # needs ~33.4 MiB of scratch
+    w = syn.Q2B_LAYER.with_seq(2048)   # needs ~76 MiB of scratch
     cfg = m.config_of(w)
     _, packed = layer_on_device(w.with_seq(8))
     x = torch.zeros((w.seq, w.hidden), dtype=torch.bfloat16, device="cuda")
