@@ -271,6 +271,316 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Two query heads per CTA (the heads 2m, 2m+1 of one KV group, same 128 query
+// rows), so every K/V tile loaded serves both. The MMA warp interleaves the
+// two heads: while softmax warpgroup A works on S_A(j) the tensor core runs
+// S_B(j), and while softmax B works the tensor core runs P_A(j) V(j) and
+// S_A(j+1). P_X(j) is written back as bf16 into the first 64 TMEM columns of
+// S_X (two per 32-bit column) and read from there as the A operand of the
+// P V product; tcgen05.mma operations of one thread run in issue order, so
+// S_X(j+1), issued after P_X(j) V(j), overwrites those columns only after
+// they were read. The running max is raised lazily: O and l are rescaled
+// only when a row's max grows by more than 2^8, so P entries stay <= 256.
+//
+// Roles (320 threads): warp 0 TMA, warp 1 MMA, warps 2-5 softmax of head A,
+// warps 6-9 softmax of head B (thread = query row).
+// TMEM: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
+// ---------------------------------------------------------------------------
+// 2^x for x <= 8 on the FMA/ALU pipes, to take part of the exponentials off
+// the special-function unit. x = i + f with i = rint(x) (through the 1.5*2^23
+// rounding constant) and f in [-0.5, 0.5]; 2^f is a cubic fitted by
+// Lawson-weighted least squares on Chebyshev nodes (near-minimax, max
+// relative error 7.5e-5, far below bf16's 2^-9 rounding); 2^i is added into
+// the exponent field. x is clamped at -125 so the result stays normal.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + 12582912.0f;
+  const float f = x - (t - 12582912.0f);
+  const float p = fmaf(fmaf(fmaf(0.0551716648f, f, 0.2426111251f), f, 0.6932609677f), f,
+                       0.9999280572f);
+  return __int_as_float(__float_as_int(p) + ((__float_as_int(t) - 0x4B400000) << 23));
+}
+
+// Row max of the raw scores in a 128-column S buffer (diagonal tile: keys
+// past the query row excluded).
+template <bool kDiag>
+__device__ __forceinline__ float row_max_raw(uint32_t tS, int r) {
+  float mx = -INFINITY;
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    uint32_t a[32], b[32];
+    tmem_ld32(tS + 64 * hh, a);
+    tmem_ld32(tS + 64 * hh + 32, b);
+    tmem_ld_wait();
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+      if (!kDiag || 64 * hh + t <= r) mx = fmaxf(mx, __uint_as_float(a[t]));
+      if (!kDiag || 64 * hh + 32 + t <= r) mx = fmaxf(mx, __uint_as_float(b[t]));
+    }
+  }
+  return mx;
+}
+
+// P = 2^(s*sc - m) for the 128 columns, written as packed bf16 pairs into the
+// first 64 TMEM columns of the same S buffer; returns the fp32 row sum. One
+// element in four goes through exp2_poly, the rest through ex2.approx.
+template <bool kDiag>
+__device__ __forceinline__ float exp_pass(uint32_t tS, int r, float sc, float m) {
+  float rs = 0.f;
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    uint32_t a[32];
+    tmem_ld32(tS + 32 * cc, a);
+    tmem_ld_wait();
+    uint32_t pk[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+      const int c0 = 32 * cc + 2 * t;
+      const float x0 = fmaf(__uint_as_float(a[2 * t]), sc, -m);
+      const float x1 = fmaf(__uint_as_float(a[2 * t + 1]), sc, -m);
+      float e0 = ex2_approx(x0);
+      float e1 = (t & 1) ? exp2_poly(x1) : ex2_approx(x1);
+      if (kDiag) {
+        if (c0 > r) e0 = 0.f;
+        if (c0 + 1 > r) e1 = 0.f;
+      }
+      rs += e0 + e1;
+      const __nv_bfloat162 b2 = __floats2bfloat162_rn(e0, e1);
+      pk[t] = *reinterpret_cast<const uint32_t*>(&b2);
+    }
+    tmem_st16(tS + 16 * cc, pk);
+  }
+  return rs;
+}
+
+constexpr int kThreads2 = 320;
+constexpr size_t kSmem2 = 1024 + 6 * size_t(kTileBytes) + 256;  // Q_A, Q_B, K[2], V[2]
+constexpr float kRescaleLog2 = 8.0f;
+
+__global__ void __launch_bounds__(kThreads2, 1)
+attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint8_t* sQ = smem;                   // [2] heads
+  uint8_t* sK = smem + 2 * kTileBytes;  // [2] stages
+  uint8_t* sV = smem + 4 * kTileBytes;  // [2] stages
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 6 * kTileBytes);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;   // [2]
+  uint64_t* k_empty = bars + 3;  // [2]
+  uint64_t* v_full = bars + 5;   // [2]
+  uint64_t* v_empty = bars + 7;  // [2]
+  uint64_t* s_full = bars + 9;   // [2] per head
+  uint64_t* p_full = bars + 11;  // [2] per head
+  uint64_t* o_final = bars + 13;
+  uint64_t* drain = bars + 14;
+  uint64_t* tok = bars + 15;     // [2]: head x finished the exponentials of a tile
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pairs = p.nh / 2;
+  const int qt = p.num_qt - 1 - static_cast<int>(blockIdx.x / pairs);
+  const int h0 = 2 * static_cast<int>(blockIdx.x % pairs);
+  const int g = h0 / (p.nh / p.nkv);
+  const int n_kv = qt + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(k_full + s, 1); mbar_init(k_empty + s, 1);
+      mbar_init(v_full + s, 1); mbar_init(v_empty + s, 1);
+      mbar_init(s_full + s, 1); mbar_init(p_full + s, 128);
+    }
+    mbar_init(o_final, 1);
+    mbar_init(drain, 1);
+    mbar_init(tok + 0, 128);
+    mbar_init(tok + 1, 128);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, 2 * kTileBytes);
+      for (int x = 0; x < 2; ++x) {
+        tma_load_2d(sQ + x * kTileBytes, &tm, q_full, (h0 + x) * 128, qt * kTile);
+        tma_load_2d(sQ + x * kTileBytes + kBlockBytes, &tm, q_full, (h0 + x) * 128 + 64,
+                    qt * kTile);
+      }
+      int nk_issued = 0, nv_issued = 0;
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        if (!mbar_wait(k_empty + s, ph ^ 1, p.err, kWhereAttnProducer, abort_flag)) break;
+        mbar_arrive_expect_tx(k_full + s, kTileBytes);
+        tma_load_2d(sK + s * kTileBytes, &tm, k_full + s, p.k_col0 + g * 128, j * kTile);
+        tma_load_2d(sK + s * kTileBytes + kBlockBytes, &tm, k_full + s, p.k_col0 + g * 128 + 64,
+                    j * kTile);
+        ++nk_issued;
+        if (!mbar_wait(v_empty + s, ph ^ 1, p.err, kWhereAttnProducer, abort_flag)) break;
+        mbar_arrive_expect_tx(v_full + s, kTileBytes);
+        tma_load_2d(sV + s * kTileBytes, &tm, v_full + s, p.v_col0 + g * 128, j * kTile);
+        tma_load_2d(sV + s * kTileBytes + kBlockBytes, &tm, v_full + s, p.v_col0 + g * 128 + 64,
+                    j * kTile);
+        ++nv_issued;
+      }
+      mbar_wait(q_full, 0, p.err, kWhereAttnDrain, nullptr);
+      for (int j = nk_issued - 2; j < nk_issued; ++j)
+        if (j >= 0) mbar_wait(k_full + (j & 1), (j >> 1) & 1, p.err, kWhereAttnDrain, nullptr);
+      for (int j = nv_issued - 2; j < nv_issued; ++j)
+        if (j >= 0) mbar_wait(v_full + (j & 1), (j >> 1) & 1, p.err, kWhereAttnDrain, nullptr);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, 128, false, true);
+      auto issue_s = [&](int x, int j) {
+        const uint32_t q0 = smem_u32(sQ + x * kTileBytes);
+        const uint32_t k0 = smem_u32(sK + (j & 1) * kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kBlockBytes + (kk & 3) * 32;
+          umma_bf16_ss(tmem + x * 128, sdesc_sw128(q0 + off, 16, 1024),
+                       sdesc_sw128(k0 + off, 16, 1024), idesc_s, kk > 0);
+        }
+        umma_commit(s_full + x);
+      };
+      auto issue_pv = [&](int x, int j) {
+        const uint32_t v0 = smem_u32(sV + (j & 1) * kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_bf16_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8,
+                       sdesc_sw128(v0 + kk * 2048, kBlockBytes, 1024), idesc_o, (j | kk) != 0);
+      };
+      bool ok = mbar_wait(q_full, 0, p.err, kWhereAttnMma, abort_flag) &&
+                mbar_wait(k_full, 0, p.err, kWhereAttnMma, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+        umma_commit(k_empty);
+      }
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const int s = j & 1;
+        const bool more = j + 1 < n_kv;
+        if (!mbar_wait(v_full + s, (j >> 1) & 1, p.err, kWhereAttnMma, abort_flag)) break;
+        if (!mbar_wait(p_full + 0, j & 1, p.err, kWhereAttnMma, abort_flag)) break;
+        tc_fence_after();
+        issue_pv(0, j);
+        if (more) {
+          if (!mbar_wait(k_full + (s ^ 1), ((j + 1) >> 1) & 1, p.err, kWhereAttnMma, abort_flag))
+            break;
+          tc_fence_after();
+          issue_s(0, j + 1);
+        }
+        if (!mbar_wait(p_full + 1, j & 1, p.err, kWhereAttnMma, abort_flag)) break;
+        tc_fence_after();
+        issue_pv(1, j);
+        umma_commit(v_empty + s);
+        if (more) {
+          issue_s(1, j + 1);
+          umma_commit(k_empty + (s ^ 1));
+        }
+      }
+      umma_commit(o_final);
+      umma_commit(drain);
+      mbar_wait(drain, 0, p.err, kWhereAttnDrain, nullptr);
+    }
+  } else {
+    const int x = (warp - 2) >> 2;  // head of this warpgroup
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_field = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + x * 128 + lane_field;
+    const uint32_t tO = tmem + 256 + x * 128 + lane_field;
+    const int64_t qpos = int64_t(qt) * kTile + r;
+    const float sc = p.scale_log2;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      ok = mbar_wait(s_full + x, j & 1, p.err, kWhereAttnSoftmax, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+      const bool diag = j == qt;
+      // pass 1: row max of the raw (unscaled) scores; the scale is positive
+      const float mx = diag ? row_max_raw<true>(tS, r) : row_max_raw<false>(tS, r);
+      const float m_new = fmaxf(m, mx * sc);
+      const bool grow = m_new > m + kRescaleLog2;
+      const float m_use = grow ? m_new : m;
+      const float alpha = grow ? ex2_approx(m - m_new) : 1.0f;
+      // the two heads take turns on the special-function unit: A(j), B(j), A(j+1), ...
+      if (x == 0) {
+        if (j > 0) ok = mbar_wait(tok + 1, (j - 1) & 1, p.err, kWhereAttnSoftmax, abort_flag);
+      } else {
+        ok = mbar_wait(tok + 0, j & 1, p.err, kWhereAttnSoftmax, abort_flag);
+      }
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      // pass 2: P = 2^(s*scale - m) as bf16 into the first 64 columns of S
+      const float rs = diag ? exp_pass<true>(tS, r, sc, m_use) : exp_pass<false>(tS, r, sc, m_use);
+      if (x == 0) mbar_arrive(tok + 0);
+      else if (j + 1 < n_kv) mbar_arrive(tok + 1);
+      l = l * alpha + rs;
+      m = m_use;
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        // O_X(j-1) is complete: S_X(j) was issued after P_X(j-1) V(j-1).
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * c, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * alpha);
+          tmem_st32(tO + 32 * c, o);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(p_full + x);
+    }
+    if (ok) {
+      ok = mbar_wait(o_final, 0, p.err, kWhereAttnSoftmax, abort_flag);
+      if (__all_sync(0xffffffffu, ok)) {
+        tc_fence_after();
+        const float inv_l = 1.0f / l;
+        __nv_bfloat16* dst = p.o + qpos * p.ldo + (h0 + x) * 128;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * c, o);
+          tmem_ld_wait();
+          if (qpos < p.S) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+              d4[t] = make_uint4(
+                  pack_bf16x2(__uint_as_float(o[8 * t]) * inv_l, __uint_as_float(o[8 * t + 1]) * inv_l),
+                  pack_bf16x2(__uint_as_float(o[8 * t + 2]) * inv_l, __uint_as_float(o[8 * t + 3]) * inv_l),
+                  pack_bf16x2(__uint_as_float(o[8 * t + 4]) * inv_l, __uint_as_float(o[8 * t + 5]) * inv_l),
+                  pack_bf16x2(__uint_as_float(o[8 * t + 6]) * inv_l, __uint_as_float(o[8 * t + 7]) * inv_l));
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_attention_tc(const q3vl_config& c, const void* qkv, int64_t S, void* o,
@@ -289,6 +599,15 @@ cudaError_t launch_attention_tc(const q3vl_config& c, const void* qkv, int64_t S
   p.ldo = q_dim(c);
   p.scale_log2 = 1.4426950408889634f / sqrtf(128.0f);
   p.err = device_error_ptr();
+  if ((p.nh / p.nkv) % 2 == 0) {
+    // two query heads of one KV group per CTA
+    cudaError_t e = cudaFuncSetAttribute(
+        attn2_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem2));
+    if (e != cudaSuccess) return e;
+    const unsigned grid = static_cast<unsigned>(int64_t(p.num_qt) * (p.nh / 2));
+    attn2_tc_kernel<<<grid, kThreads2, kSmem2, st>>>(tm, p);
+    return counted_launch(1);
+  }
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmem));
   if (e != cudaSuccess) return e;
