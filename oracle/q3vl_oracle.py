@@ -290,27 +290,32 @@ def _np(t, dtype):
     return np.asarray(t, dtype=dtype)
 
 
-def qkv(cfg: Config, W: Dict, x: np.ndarray, angles: np.ndarray, dtype=np.float64):
+def qkv(cfg: Config, W: Dict, x: np.ndarray, angles: np.ndarray, dtype=np.float64,
+        q_rows: Optional[np.ndarray] = None):
     """Steps up to the attention inputs: norm, projections (+bias), q/k norm, MRoPE.
 
     Returns q [S, nh, hd], k [S, nkv, hd], v [S, nkv, hd]. The bias is added
     right after the projection and before the per-head norm (hf2q
     ``qwen3vl_text/forward.rs`` module doc); the per-head norm comes before
-    the rotation (``Qwen3Encoder::norm_rope``).
+    the rotation (``Qwen3Encoder::norm_rope``). With ``q_rows`` only those
+    rows of q are formed (the others stay zero); k and v always cover every row.
     """
     S = x.shape[0]
     hd, nh, nkv = cfg.head_dim, cfg.n_heads, cfg.n_kv_heads
+    qr = np.arange(S) if q_rows is None else np.asarray(q_rows)
     xn = rms_norm(x, _np(W["attn_norm"], dtype), cfg.rms_eps)
-    q = xn @ _np(W["wq"], dtype).T
+    q = xn[qr] @ _np(W["wq"], dtype).T
     k = xn @ _np(W["wk"], dtype).T
     v = xn @ _np(W["wv"], dtype).T
     if W.get("bq") is not None:
         q = q + _np(W["bq"], dtype)
         k = k + _np(W["bk"], dtype)
         v = v + _np(W["bv"], dtype)
-    q = rms_norm(q.reshape(S, nh, hd), _np(W["q_norm"], dtype), cfg.rms_eps)
+    q = rms_norm(q.reshape(len(qr), nh, hd), _np(W["q_norm"], dtype), cfg.rms_eps)
     k = rms_norm(k.reshape(S, nkv, hd), _np(W["k_norm"], dtype), cfg.rms_eps)
-    return rope_rotate(q, angles), rope_rotate(k, angles), v.reshape(S, nkv, hd)
+    q_all = np.zeros((S, nh, hd), dtype=q.dtype)
+    q_all[qr] = rope_rotate(q, angles[qr])
+    return q_all, rope_rotate(k, angles), v.reshape(S, nkv, hd)
 
 
 def o_residual(W: Dict, o: np.ndarray, x: np.ndarray, dtype=np.float64) -> np.ndarray:
@@ -345,9 +350,9 @@ def layer(cfg: Config, W: Dict, x, pos: np.ndarray, ds_slab=None, ds_rows=None,
     S = x.shape[0]
     nh, hd = cfg.n_heads, cfg.head_dim
     angles = mrope_angles(pos, cfg.rope_theta, hd, cfg.mrope_section)
-    q, k, v = qkv(cfg, W, x, angles, dtype)
-    o = attention(q, k, v, rows)
     sel = np.arange(S) if rows is None else np.asarray(rows)
+    q, k, v = qkv(cfg, W, x, angles, dtype, None if rows is None else sel)
+    o = attention(q, k, v, rows)
     h = np.zeros_like(x)
     h[sel] = o_residual(W, o[sel].reshape(len(sel), nh * hd), x[sel], dtype)
     a = ffn_act(cfg, W, h[sel], dtype)

@@ -66,18 +66,20 @@ struct Params {
   int32_t* sk_flags;
 };
 
-// Work schedule shared by the three roles of a CTA.
+// Work schedule shared by the three roles of a CTA. Each CTA first works
+// through its stream-K range, then its data-parallel tiles:
 //   tiles [0, dp_tiles): data parallel; CTA c takes tiles c, c + G, ... over
 //     their whole K range;
 //   tiles [dp_tiles, T): stream-K; their U = (T - dp_tiles) * KB k-block
 //     units are cut into G equal contiguous ranges, CTA c taking units
 //     [c U / G, (c + 1) U / G).
 // A stream-K tile split across CTAs is finished by the CTA holding its first
-// k-block, which reaches it last in time (at the end of its range). The CTAs
-// holding its later k-blocks reach them first (at the start of their
+// k-block, which reaches it last (at the end of its stream-K range). The
+// CTAs holding its later k-blocks reach them first (at the start of their
 // ranges): they leave fp32 partial sums in their own scratch slot and raise
 // their flag; the finisher adds the partials in CTA order (deterministic)
-// before the fused epilogue.
+// before the fused epilogue. Running the stream-K part first lets these
+// longer epilogues overlap the data-parallel main loops that follow.
 enum Role : int { kFull = 0, kFinisher = 1, kContributor = 2 };
 
 struct Work {
@@ -93,20 +95,22 @@ struct WorkIter {
       : dp_t(c), dp_tiles(p.dp_tiles), stride(G), u(p.sk_units * c / G),
         u1(p.sk_units * (c + 1) / G), sk_base(p.dp_tiles), KB(p.kb_per_tile) {}
   __device__ bool next(Work& w) {
+    if (u < u1) {
+      const int64_t t = u / KB;
+      const int64_t end = min(u1, (t + 1) * KB);
+      w.tile = sk_base + t;
+      w.kb0 = static_cast<int>(u - t * KB);
+      w.kb1 = static_cast<int>(end - t * KB);
+      w.role = w.kb0 > 0 ? kContributor : (w.kb1 == KB ? kFull : kFinisher);
+      u = end;
+      return true;
+    }
     if (dp_t < dp_tiles) {
       w.tile = dp_t; w.kb0 = 0; w.kb1 = KB; w.role = kFull;
       dp_t += stride;
       return true;
     }
-    if (u >= u1) return false;
-    const int64_t t = u / KB;
-    const int64_t end = min(u1, (t + 1) * KB);
-    w.tile = sk_base + t;
-    w.kb0 = static_cast<int>(u - t * KB);
-    w.kb1 = static_cast<int>(end - t * KB);
-    w.role = w.kb0 > 0 ? kContributor : (w.kb1 == KB ? kFull : kFinisher);
-    u = end;
-    return true;
+    return false;
   }
 };
 
@@ -133,14 +137,28 @@ __device__ __forceinline__ void epilogue_sync() { asm volatile("barrier.sync 1, 
 template <int BN>
 __device__ __forceinline__ void load_chunk(uint32_t taddr, int cc, int rr, const float* part,
                                            int n_part, float* v) {
+  // the first contributor's partial is requested before the TMEM load so the
+  // two latencies overlap
+  float4 q0[8];
+  const size_t off = (static_cast<size_t>(cc) * BM + rr) * 32;
+  if (n_part > 0) {
+    const float4* src = reinterpret_cast<const float4*>(part + off);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) q0[j] = __ldcg(src + j);
+  }
   uint32_t r[32];
   tmem_ld32(taddr, r);
   tmem_ld_wait();
 #pragma unroll
   for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(r[t]);
-  for (int i = 0; i < n_part; ++i) {
-    const float4* src = reinterpret_cast<const float4*>(
-        part + static_cast<size_t>(i) * (BM * BN) + (static_cast<size_t>(cc) * BM + rr) * 32);
+  if (n_part > 0) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      v[4 * j] += q0[j].x; v[4 * j + 1] += q0[j].y; v[4 * j + 2] += q0[j].z; v[4 * j + 3] += q0[j].w;
+    }
+  }
+  for (int i = 1; i < n_part; ++i) {
+    const float4* src = reinterpret_cast<const float4*>(part + static_cast<size_t>(i) * (BM * BN) + off);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const float4 q = __ldcg(src + j);
@@ -407,17 +425,39 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             }
           }
         } else {
-          const int32_t dsk =
-              (EPI == static_cast<int>(Epi::kResidual) && valid && p.ds_map != nullptr)
-                  ? p.ds_map[row] : -1;
+          constexpr bool kRes = EPI == static_cast<int>(Epi::kResidual);
+          const int32_t dsk = (kRes && valid && p.ds_map != nullptr) ? p.ds_map[row] : -1;
+          // residual chunks are requested one chunk ahead of their use
+          uint4 res[4];
+          const uint4* rsrc = reinterpret_cast<const uint4*>(p.resid + row * p.ldo + n0);
+          if (kRes && valid) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) res[j] = __ldg(rsrc + j);
+          }
 #pragma unroll 1
           for (int cc = 0; cc < BN / 32; ++cc) {
+            uint4 cur[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) cur[j] = res[j];
+            if (kRes && valid && cc + 1 < BN / 32) {
+#pragma unroll
+              for (int j = 0; j < 4; ++j) res[j] = __ldg(rsrc + 4 * (cc + 1) + j);
+            }
             float v[32];
             load_chunk<BN>(tbase + 32 * cc, cc, rr, part, n_part, v);
             if (valid) {
               const int64_t col = n0 + 32 * cc;
-              if constexpr (EPI == static_cast<int>(Epi::kResidual)) {
-                add_bf16x32(v, p.resid + row * p.ldo + col);
+              if constexpr (kRes) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const uint32_t wds[4] = {cur[j].x, cur[j].y, cur[j].z, cur[j].w};
+#pragma unroll
+                  for (int t = 0; t < 4; ++t) {
+                    const float2 f = unpack_bf16x2(wds[t]);
+                    v[8 * j + 2 * t] += f.x;
+                    v[8 * j + 2 * t + 1] += f.y;
+                  }
+                }
                 if (dsk >= 0) add_bf16x32(v, p.ds_slab + int64_t(dsk) * p.N + col);
               }
               store_bf16x32(p.out + row * p.ldo + col, v);
