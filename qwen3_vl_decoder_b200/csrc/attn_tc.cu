@@ -302,43 +302,32 @@ __device__ __forceinline__ float exp2_poly(float x) {
   return __int_as_float(__float_as_int(p) + ((__float_as_int(t) - 0x4B400000) << 23));
 }
 
-// Row max of the raw scores in a 128-column S buffer (diagonal tile: keys
-// past the query row excluded).
+// Row max of the raw (unscaled) scores of one 128-column tile held in
+// registers (diagonal tile: keys past the query row excluded).
 template <bool kDiag>
-__device__ __forceinline__ float row_max_raw(uint32_t tS, int r) {
+__device__ __forceinline__ float row_max_regs(const uint32_t* sr, int r) {
   float mx = -INFINITY;
 #pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    uint32_t a[32], b[32];
-    tmem_ld32(tS + 64 * hh, a);
-    tmem_ld32(tS + 64 * hh + 32, b);
-    tmem_ld_wait();
-#pragma unroll
-    for (int t = 0; t < 32; ++t) {
-      if (!kDiag || 64 * hh + t <= r) mx = fmaxf(mx, __uint_as_float(a[t]));
-      if (!kDiag || 64 * hh + 32 + t <= r) mx = fmaxf(mx, __uint_as_float(b[t]));
-    }
-  }
+  for (int c = 0; c < 128; ++c)
+    if (!kDiag || c <= r) mx = fmaxf(mx, __uint_as_float(sr[c]));
   return mx;
 }
 
-// P = 2^(s*sc - m) for the 128 columns, written as packed bf16 pairs into the
-// first 64 TMEM columns of the same S buffer; returns the fp32 row sum. One
-// element in four goes through exp2_poly, the rest through ex2.approx.
+// P = 2^(s*sc - m) for the 128 columns of a score row held in registers,
+// written as packed bf16 pairs into the first 64 TMEM columns of the same S
+// buffer; returns the fp32 row sum. One element in four goes through
+// exp2_poly, the rest through ex2.approx.
 template <bool kDiag>
-__device__ __forceinline__ float exp_pass(uint32_t tS, int r, float sc, float m) {
+__device__ __forceinline__ float exp_regs(const uint32_t* sr, uint32_t tS, int r, float sc, float m) {
   float rs = 0.f;
 #pragma unroll
   for (int cc = 0; cc < 4; ++cc) {
-    uint32_t a[32];
-    tmem_ld32(tS + 32 * cc, a);
-    tmem_ld_wait();
     uint32_t pk[16];
 #pragma unroll
     for (int t = 0; t < 16; ++t) {
       const int c0 = 32 * cc + 2 * t;
-      const float x0 = fmaf(__uint_as_float(a[2 * t]), sc, -m);
-      const float x1 = fmaf(__uint_as_float(a[2 * t + 1]), sc, -m);
+      const float x0 = fmaf(__uint_as_float(sr[c0]), sc, -m);
+      const float x1 = fmaf(__uint_as_float(sr[c0 + 1]), sc, -m);
       float e0 = ex2_approx(x0);
       float e1 = (t & 1) ? exp2_poly(x1) : ex2_approx(x1);
       if (kDiag) {
@@ -513,8 +502,13 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
       const bool diag = j == qt;
-      // pass 1: row max of the raw (unscaled) scores; the scale is positive
-      const float mx = diag ? row_max_raw<true>(tS, r) : row_max_raw<false>(tS, r);
+      // the whole score row in registers: one batch of TMEM loads, one wait
+      uint32_t sr[128];
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) tmem_ld32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(sr + 32 * cc));
+      tmem_ld_wait();
+      // row max of the raw (unscaled) scores; the scale is positive
+      const float mx = diag ? row_max_regs<true>(sr, r) : row_max_regs<false>(sr, r);
       const float m_new = fmaxf(m, mx * sc);
       const bool grow = m_new > m + kRescaleLog2;
       const float m_use = grow ? m_new : m;
@@ -527,7 +521,7 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
       }
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       // pass 2: P = 2^(s*scale - m) as bf16 into the first 64 columns of S
-      const float rs = diag ? exp_pass<true>(tS, r, sc, m_use) : exp_pass<false>(tS, r, sc, m_use);
+      const float rs = diag ? exp_regs<true>(sr, tS, r, sc, m_use) : exp_regs<false>(sr, tS, r, sc, m_use);
       if (x == 0) mbar_arrive(tok + 0);
       else if (j + 1 < n_kv) mbar_arrive(tok + 1);
       l = l * alpha + rs;

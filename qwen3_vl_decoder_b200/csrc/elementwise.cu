@@ -182,6 +182,9 @@ cudaError_t launch_positions(const uint8_t* tt, int64_t S, const int32_t* grids,
 // ---------------------------------------------------------------------------
 __global__ void rope_table_kernel(const int32_t* __restrict__ pos, int64_t S, double theta,
                                   int sec_h, int sec_w, float2* __restrict__ cs) {
+  __shared__ double freq[kHalf];
+  if (threadIdx.x < kHalf) freq[threadIdx.x] = pow(theta, -2.0 * threadIdx.x / kHeadDim);
+  __syncthreads();
   const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= S * kHalf) return;
   const int64_t p = idx / kHalf;
@@ -189,8 +192,7 @@ __global__ void rope_table_kernel(const int32_t* __restrict__ pos, int64_t S, do
   int axis = 0;
   if (i % 3 == 1 && i < 3 * sec_h) axis = 1;
   else if (i % 3 == 2 && i < 3 * sec_w) axis = 2;
-  const double freq = pow(theta, -2.0 * i / kHeadDim);
-  const double ang = static_cast<double>(pos[axis * S + p]) * freq;
+  const double ang = static_cast<double>(pos[axis * S + p]) * freq[i];
   double s, c;
   sincos(ang, &s, &c);
   cs[idx] = make_float2(static_cast<float>(c), static_cast<float>(s));

@@ -70,6 +70,7 @@ struct Params {
   // schedule over pair tiles (see WorkIter)
   int64_t dp_tiles, sk_units;
   int kb_per_tile;
+  int m_fastest;  // tile order: 1 = M index fastest (A stays in L2), 0 = N fastest (B stays)
   // stream-K scratch: one fp32 128 x BN partial tile and one flag per CTA
   float* sk_partials;
   int32_t* sk_flags;
@@ -123,6 +124,13 @@ struct WorkIter {
     return false;
   }
 };
+
+// Row-tile and column-tile index of pair tile t.
+__device__ __forceinline__ void tile_mn(const Params& p, int64_t t, int64_t num_m, int64_t num_n,
+                                        int64_t& m, int64_t& n) {
+  if (p.m_fastest) { m = t % num_m; n = t / num_m; }
+  else { n = t % num_n; m = t / num_n; }
+}
 
 // Owner pair of stream-K unit u: the largest c with c U / G <= u.
 __device__ __forceinline__ int sk_owner(int64_t u, int64_t U, int G) {
@@ -322,6 +330,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const uint32_t tmem_base = *tmem_slot;
 
   const int64_t num_m = (p.M + 2 * BM - 1) / (2 * BM);
+  const int64_t num_n = p.N / BN;
   const int G = static_cast<int>(gridDim.x >> 1);
   const int c = static_cast<int>(blockIdx.x >> 1);
 
@@ -334,8 +343,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       Work w;
       bool ok = true;
       while (ok && it.next(w)) {
-        const int32_t m0 = static_cast<int32_t>((w.tile % num_m) * 2 * BM + rank * BM);
-        const int32_t n0 = static_cast<int32_t>((w.tile / num_m) * BN + rank * (BN / 2));
+        int64_t tm, tn;
+        tile_mn(p, w.tile, num_m, num_n, tm, tn);
+        const int32_t m0 = static_cast<int32_t>(tm * 2 * BM + rank * BM);
+        const int32_t n0 = static_cast<int32_t>(tn * BN + rank * (BN / 2));
         for (int kb = w.kb0; kb < w.kb1; ++kb) {
           if (!mbar_wait(empty + stage, ph ^ 1, p.err, kWhereGemmProducer, abort_flag)) {
             ok = false;
@@ -411,9 +422,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     Work w;
     while (it.next(w)) {
       const int buf = acc_i & 1;
-      const int64_t row0 = (w.tile % num_m) * 2 * BM + rank * BM;
+      int64_t tm, tn;
+      tile_mn(p, w.tile, num_m, num_n, tm, tn);
+      const int64_t row0 = tm * 2 * BM + rank * BM;
       const int64_t row = row0 + rr;
-      const int64_t n0 = (w.tile / num_m) * BN;
+      const int64_t n0 = tn * BN;
       const bool valid = row < p.M;
       const bool stores = w.role != kContributor;
       // the epilogue tile is free once the previous TMA store has read it
@@ -559,7 +572,7 @@ HostSched make_sched(int64_t tiles, int kb, int max_pairs) {
   HostSched h{};
   const int64_t waves = (tiles + max_pairs - 1) / max_pairs;
   const double dp_eff = static_cast<double>(tiles) / static_cast<double>(waves * max_pairs);
-  if (dp_eff >= 0.9) {
+  if (dp_eff >= 0.85) {
     h.pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
     h.dp_tiles = tiles;
     h.sk_units = 0;
@@ -621,6 +634,8 @@ cudaError_t launch_bn(const GemmArgs& a, Params p, cudaStream_t st) {
   p.dp_tiles = h.dp_tiles;
   p.sk_units = h.sk_units;
   p.kb_per_tile = static_cast<int>(a.K / BK);
+  // keep the smaller operand resident in L2 while the larger one streams
+  p.m_fastest = a.M <= a.N ? 1 : 0;
   kern<<<grid, kThreads, C::kSmem, st>>>(tmA, tmB, tmOut, tmRes, p);
   return counted_launch(1);
 }
