@@ -12,7 +12,8 @@ needed between steps.
   value     tokens/s per layer, inputs resident in HBM, CUDA events on the
             launching stream, max over ranks;
   e2e       the same through the public API with host buffers: pinned x and
-            token types copied in, x' copied out, every step;
+            token types copied in, x' copied out, every step (uploads and
+            downloads on their own streams, overlapping other steps' kernels);
   roofline  the dominant kernel (gate/up GEMM with SiLU*up epilogue), timed
             live by stage events the library records inside the timed steps;
   cpu_baseline the CPU oracle (fp32 NumPy) on a bounded sample.
@@ -179,15 +180,54 @@ def device_step(st, events=None):
     q3.layer_prefill(st["cfg"], st["packed"], st["x"], pos, st["slab"], st["rows"], st["ws"])
 
 
-def e2e_step(st):
-    q3 = st["q3"]
-    st["x"].copy_(st["x_host"], non_blocking=True)
-    st["tt"].copy_(st["tt_host"], non_blocking=True)
-    if st["g"] is not None:
-        st["g"].copy_(st["g_host"], non_blocking=True)
-    pos, _ = q3.mrope_positions(st["tt"], st["g"], check=False)
-    q3.layer_prefill(st["cfg"], st["packed"], st["x"], pos, st["slab"], st["rows"], st["ws"])
-    st["out_host"].copy_(st["x"], non_blocking=True)
+class E2EPipeline:
+    """End-to-end steps through the public API with host buffers.
+
+    Every step copies its inputs (x, token types, grids) from pinned host
+    memory to the device, runs P0..P9, and copies x' back to pinned host
+    memory. Uploads, compute and downloads run on three streams with
+    double-buffered device inputs, so step k+1's upload and step k-1's
+    download overlap step k's kernels, as a serving loop would.
+    """
+
+    def __init__(self, st, dev):
+        self.st = st
+        self.s_in = torch.cuda.Stream(dev)
+        self.s_out = torch.cuda.Stream(dev)
+        self.s_comp = torch.cuda.current_stream(dev)
+        self.x = [st["x"], torch.empty_like(st["x"])]
+        self.tt = [st["tt"], torch.empty_like(st["tt"])]
+        self.g = [st["g"], None if st["g"] is None else torch.empty_like(st["g"])]
+        self.out = [st["out_host"], torch.empty_like(st["out_host"]).pin_memory()]
+        self.in_done = [torch.cuda.Event() for _ in range(2)]
+        self.comp_done = [torch.cuda.Event() for _ in range(2)]
+        self.out_done = [torch.cuda.Event() for _ in range(2)]
+        self.started = [False, False]
+
+    def step(self, k):
+        st, q3, b = self.st, self.st["q3"], k % 2
+        with torch.cuda.stream(self.s_in):
+            if self.started[b]:
+                self.s_in.wait_event(self.out_done[b])   # x[b] was read by its download
+            self.x[b].copy_(st["x_host"], non_blocking=True)
+            self.tt[b].copy_(st["tt_host"], non_blocking=True)
+            if self.g[b] is not None:
+                self.g[b].copy_(st["g_host"], non_blocking=True)
+            self.in_done[b].record(self.s_in)
+        self.s_comp.wait_event(self.in_done[b])
+        pos, _ = q3.mrope_positions(self.tt[b], self.g[b], check=False, stream=self.s_comp)
+        q3.layer_prefill(st["cfg"], st["packed"], self.x[b], pos, st["slab"], st["rows"], st["ws"],
+                         stream=self.s_comp)
+        self.comp_done[b].record(self.s_comp)
+        with torch.cuda.stream(self.s_out):
+            self.s_out.wait_event(self.comp_done[b])
+            self.out[b].copy_(self.x[b], non_blocking=True)
+            self.out_done[b].record(self.s_out)
+        self.started[b] = True
+
+    def finish(self):
+        self.s_comp.wait_stream(self.s_in)
+        self.s_comp.wait_stream(self.s_out)
 
 
 def barrier(world):
@@ -309,9 +349,20 @@ def main():
                 for i, name in enumerate(STAGES)}
 
     # end-to-end through the public API with host buffers
-    for _ in range(3):
-        e2e_step(st)
-    t_e2e = timed(lambda k: e2e_step(st), args.steps, world, dev)
+    pipe = E2EPipeline(st, dev)
+    for k in range(3):
+        pipe.step(k)
+    pipe.finish()
+
+    def e2e_steps(k):
+        if k == 0:   # the copy streams start after the timed region's start event
+            pipe.s_in.wait_stream(pipe.s_comp)
+            pipe.s_out.wait_stream(pipe.s_comp)
+        pipe.step(k)
+        if k == args.steps - 1:
+            pipe.finish()   # the timed region ends after the last download
+
+    t_e2e = timed(e2e_steps, args.steps, world, dev)
     q3.check_device()
     assert torch.isfinite(st["out_host"].float()).all(), "non-finite output"
 

@@ -287,60 +287,63 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
 // warps 6-9 softmax of head B (thread = query row).
 // TMEM: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
 // ---------------------------------------------------------------------------
-// 2^x for x <= 8 on the FMA/ALU pipes, to take part of the exponentials off
-// the special-function unit. x = i + f with i = rint(x) (through the 1.5*2^23
-// rounding constant) and f in [-0.5, 0.5]; 2^f is a cubic fitted by
-// Lawson-weighted least squares on Chebyshev nodes (near-minimax, max
-// relative error 7.5e-5, far below bf16's 2^-9 rounding); 2^i is added into
-// the exponent field. x is clamped at -125 so the result stays normal.
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -125.0f);
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  const float p = fmaf(fmaf(fmaf(0.0551716648f, f, 0.2426111251f), f, 0.6932609677f), f,
-                       0.9999280572f);
-  return __int_as_float(__float_as_int(p) + ((__float_as_int(t) - 0x4B400000) << 23));
-}
-
 // Row max of the raw (unscaled) scores of one 128-column tile held in
 // registers (diagonal tile: keys past the query row excluded).
 template <bool kDiag>
 __device__ __forceinline__ float row_max_regs(const uint32_t* sr, int r) {
   float mx = -INFINITY;
+  if (kDiag) {
 #pragma unroll
-  for (int c = 0; c < 128; ++c)
-    if (!kDiag || c <= r) mx = fmaxf(mx, __uint_as_float(sr[c]));
+    for (int c = 0; c < 128; ++c)
+      if (c <= r) mx = fmaxf(mx, __uint_as_float(sr[c]));
+  } else {
+    // eight independent partial maxima keep the dependency chains short
+    float pm[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) pm[q] = fmaxf(__uint_as_float(sr[q]), __uint_as_float(sr[q + 8]));
+#pragma unroll
+    for (int c = 16; c < 128; c += 16)
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        pm[q] = fmax3(pm[q], __uint_as_float(sr[c + q]), __uint_as_float(sr[c + q + 8]));
+    mx = fmaxf(fmaxf(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5])), fmaxf(pm[6], pm[7]));
+  }
   return mx;
 }
 
 // P = 2^(s*sc - m) for the 128 columns of a score row held in registers,
 // written as packed bf16 pairs into the first 64 TMEM columns of the same S
-// buffer; returns the fp32 row sum. One element in four goes through
-// exp2_poly, the rest through ex2.approx.
+// buffer; returns the fp32 row sum. The scale-and-shift and the running sum
+// run as packed f32x2 operations, the exponentials on ex2.approx: the
+// softmax is bound by instruction issue, not by the special-function unit.
 template <bool kDiag>
 __device__ __forceinline__ float exp_regs(const uint32_t* sr, uint32_t tS, int r, float sc, float m) {
-  float rs = 0.f;
+  const uint64_t sc2 = f2_pack(sc, sc), nm2 = f2_pack(-m, -m);
+  uint64_t acc[4];  // four independent running sums of pairs
+#pragma unroll
+  for (int q = 0; q < 4; ++q) acc[q] = f2_pack(0.f, 0.f);
 #pragma unroll
   for (int cc = 0; cc < 4; ++cc) {
     uint32_t pk[16];
 #pragma unroll
     for (int t = 0; t < 16; ++t) {
       const int c0 = 32 * cc + 2 * t;
-      const float x0 = fmaf(__uint_as_float(sr[c0]), sc, -m);
-      const float x1 = fmaf(__uint_as_float(sr[c0 + 1]), sc, -m);
-      float e0 = ex2_approx(x0);
-      float e1 = (t & 1) ? exp2_poly(x1) : ex2_approx(x1);
+      float x0, x1;
+      f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c0]), __uint_as_float(sr[c0 + 1])), sc2, nm2), x0, x1);
+      float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
       if (kDiag) {
         if (c0 > r) e0 = 0.f;
         if (c0 + 1 > r) e1 = 0.f;
       }
-      rs += e0 + e1;
+      acc[t & 3] = f2_add(acc[t & 3], f2_pack(e0, e1));
       const __nv_bfloat162 b2 = __floats2bfloat162_rn(e0, e1);
       pk[t] = *reinterpret_cast<const uint32_t*>(&b2);
     }
     tmem_st16(tS + 16 * cc, pk);
   }
-  return rs;
+  float a0, a1;
+  f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
+  return a0 + a1;
 }
 
 constexpr int kThreads2 = 320;

@@ -28,7 +28,7 @@
 //             q_norm / k_norm gain, then split-half MRoPE from the cos/sin
 //             table; v heads: v only.
 //   kResidual out = resid + acc (+ DeepStack slab row ds_map[r]).
-//   kSwiGLU   out = silu(s*g) * (s*u), s = inv_rms[r]; B's 256-row block
+//   kSwiGLU   out = silu(s*g) * (s*u), s = inv_rms[r] (fast exp / divide); B's 256-row block
 //             holds 128 gate rows then the 128 matching up rows.
 //   kPlain    out = acc.
 #include "q3vl_device.cuh"
@@ -514,7 +514,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             load_chunk<BN>(tbase + 128 + 32 * cc, cc + 4, rr, part, n_part, slot_stride, u);
             float v[32];
 #pragma unroll
-            for (int t = 0; t < 32; ++t) v[t] = silu_f(g[t] * s) * (u[t] * s);
+            for (int t = 0; t < 32; ++t) v[t] = silu_fast(g[t] * s) * (u[t] * s);
             stage_bf16x32(tile, rr, cc, v);
           }
         } else {
