@@ -255,10 +255,11 @@ def timed(fn, steps, world, dev):
     return max_over_ranks(a.elapsed_time(b) / 1e3, world, dev)
 
 
-def cpu_oracle_rate(w, seconds=10.0, min_reps=1, max_reps=1000, reps=None):
-    """tokens/s of the fp32 NumPy oracle on the first CPU_SAMPLE_TOKENS tokens of w."""
+def cpu_oracle_rate(w, seconds=10.0, min_reps=1, max_reps=1000, reps=None,
+                    tokens=CPU_SAMPLE_TOKENS):
+    """tokens/s of the fp32 NumPy oracle on the first `tokens` tokens of w."""
     from oracle import q3vl_oracle as O
-    n = min(CPU_SAMPLE_TOKENS, w.seq)
+    n = min(tokens, w.seq)
     ws = w.with_seq(n, images=tuple(im for im in w.images if im[0] + im[1] * im[2] <= n))
     raw = syn.layer_weights(ws, 0)
     x = syn.hidden_input(ws).float().numpy()
@@ -290,8 +291,15 @@ def reference_arm(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    n, warm = cpu_oracle_rate(w, reps=max(1, args.warmup))
-    n, times = cpu_oracle_rate(w, reps=max(1, args.steps))
+    # size the per-step sample so that the whole run takes about a minute
+    total = max(1, args.warmup) + max(1, args.steps)
+    tokens = 64
+    _, t64 = cpu_oracle_rate(w, reps=2, tokens=64)
+    for cand in (128, 256, 512):
+        if min(t64) * cand / 64 * total <= 90.0:
+            tokens = cand
+    n, warm = cpu_oracle_rate(w, reps=max(1, args.warmup), tokens=tokens)
+    n, times = cpu_oracle_rate(w, reps=max(1, args.steps), tokens=tokens)
     total = sum(times)
     rate = n * len(times) / total
     sample = (f"first {n} tokens of {w.name} ({w.seq} tokens), one fp32 NumPy layer pass per "

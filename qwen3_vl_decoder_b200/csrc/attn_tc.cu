@@ -367,8 +367,7 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
   uint64_t* p_full = bars + 11;  // [2] per head
   uint64_t* o_final = bars + 13;
   uint64_t* drain = bars + 14;
-  uint64_t* tok = bars + 15;     // [2]: head x finished the exponentials of a tile
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -387,8 +386,6 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
     }
     mbar_init(o_final, 1);
     mbar_init(drain, 1);
-    mbar_init(tok + 0, 128);
-    mbar_init(tok + 1, 128);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm);
@@ -516,17 +513,8 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
       const bool grow = m_new > m + kRescaleLog2;
       const float m_use = grow ? m_new : m;
       const float alpha = grow ? ex2_approx(m - m_new) : 1.0f;
-      // the two heads take turns on the special-function unit: A(j), B(j), A(j+1), ...
-      if (x == 0) {
-        if (j > 0) ok = mbar_wait(tok + 1, (j - 1) & 1, p.err, kWhereAttnSoftmax, abort_flag);
-      } else {
-        ok = mbar_wait(tok + 0, j & 1, p.err, kWhereAttnSoftmax, abort_flag);
-      }
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       // pass 2: P = 2^(s*scale - m) as bf16 into the first 64 columns of S
       const float rs = diag ? exp_regs<true>(sr, tS, r, sc, m_use) : exp_regs<false>(sr, tS, r, sc, m_use);
-      if (x == 0) mbar_arrive(tok + 0);
-      else if (j + 1 < n_kv) mbar_arrive(tok + 1);
       l = l * alpha + rs;
       m = m_use;
       if (j > 0 && __any_sync(0xffffffffu, grow)) {

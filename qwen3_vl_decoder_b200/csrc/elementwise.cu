@@ -234,17 +234,33 @@ __device__ __forceinline__ float sumsq16<__nv_bfloat16>(const uint4& v) {
   return s;
 }
 
+// Sum of squares of one row, read by a warp in batches of 8 16-byte vectors
+// per lane, all requested before any is used so the loads overlap.
+template <typename T>
+__device__ __forceinline__ float row_sumsq(const uint4* __restrict__ p, int64_t nvec, int lane) {
+  constexpr int kBatch = 8;
+  float s = 0.f;
+  for (int64_t base = 0; base < nvec; base += 32 * kBatch) {
+    uint4 v[kBatch];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const int64_t i = base + b * 32 + lane;
+      v[b] = i < nvec ? __ldg(p + i) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) s += sumsq16<T>(v[b]);
+  }
+  return warp_sum(s);
+}
+
 template <typename T>
 __global__ void rowstat_kernel(const T* __restrict__ x, int64_t S, int64_t width, float eps,
                                float* __restrict__ inv) {
   const int64_t row = int64_t(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= S) return;
-  const uint4* p = reinterpret_cast<const uint4*>(x + row * width);
-  const int64_t nvec = width * sizeof(T) / 16;
-  float s = 0.f;
-  for (int64_t v = lane; v < nvec; v += 32) s += sumsq16<T>(__ldg(p + v));
-  s = warp_sum(s);
+  const float s = row_sumsq<T>(reinterpret_cast<const uint4*>(x + row * width),
+                               width * int64_t(sizeof(T)) / 16, lane);
   if (lane == 0) inv[row] = 1.0f / sqrtf(s / static_cast<float>(width) + eps);
 }
 
@@ -294,10 +310,9 @@ __global__ void final_norm_kernel(T* __restrict__ x, int64_t S, int64_t width, f
   uint4* p = reinterpret_cast<uint4*>(x + row * width);
   const uint4* g = reinterpret_cast<const uint4*>(gain);
   const int64_t nvec = width * sizeof(T) / 16;
-  float s = 0.f;
-  for (int64_t v = lane; v < nvec; v += 32) s += sumsq16<T>(p[v]);
-  s = warp_sum(s);
+  const float s = row_sumsq<T>(p, nvec, lane);
   const float inv = 1.0f / sqrtf(s / static_cast<float>(width) + eps);
+#pragma unroll 4
   for (int64_t v = lane; v < nvec; v += 32) p[v] = scale16(p[v], inv, __ldg(g + v), T());
 }
 
