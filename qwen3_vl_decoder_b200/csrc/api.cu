@@ -68,6 +68,7 @@ WsLayout ws_layout(const q3vl_config& c, int64_t S) {
   L.h = take(size_t(S) * c.hidden * e);
   L.act = take(size_t(S) * c.intermediate * e);
   if (c.dtype == Q3VL_DTYPE_BF16) {
+    L.rowsq = take(size_t(S) * (c.hidden / 128) * sizeof(float));
     L.sk_slots = sm_count();
     L.sk_part = take(size_t(L.sk_slots) * kSkSlotBytes);
     L.sk_flags = take(size_t(L.sk_slots) * sizeof(int32_t));
@@ -259,22 +260,33 @@ int run_attention(const q3vl_config& c, const void* qkv, int64_t S, void* o, cud
                     "attention");
 }
 
+// Number of per-row sum-of-squares partials the o-projection leaves for the
+// gate/up epilogue: one per N tile of the residual GEMM.
+int rowsq_parts(const q3vl_config& c) { return c.hidden % 256 == 0 ? c.hidden / 256 : c.hidden / 128; }
+
 int run_oproj(const q3vl_config& c, const q3vl_layer& w, const void* o, const void* x, int64_t S,
-              void* h, const Sk& sk, cudaStream_t st) {
+              void* h, const Sk& sk, cudaStream_t st, float* rowsq = nullptr) {
   GemmArgs a{};
   a.A = o; a.B = w.w_o; a.M = S; a.N = c.hidden; a.K = q_dim(c);
   a.out = h; a.ldo = c.hidden; a.resid = x;
+  a.rowsq_out = rowsq;
+  a.rowsq_n = rowsq_parts(c);
   set_sk(a, sk);
   if (is_bf16(c)) return cuda_check(launch_gemm_tc(Epi::kResidual, a, st), "o projection");
   return cuda_check(launch_gemm_f32(Epi::kResidual, a, st), "o projection");
 }
 
 int run_gateup(const q3vl_config& c, const q3vl_layer& w, const void* h, int64_t S,
-               const float* inv2, void* act, const Sk& sk, cudaStream_t st) {
+               const float* inv2, void* act, const Sk& sk, cudaStream_t st,
+               const float* rowsq = nullptr) {
   if (is_bf16(c)) {
     GemmArgs a{};
     a.A = h; a.B = w.w_gu; a.M = S; a.N = 2 * int64_t(c.intermediate); a.K = c.hidden;
     a.out = act; a.ldo = c.intermediate; a.row_scale = inv2;
+    a.rowsq_in = rowsq;
+    a.rowsq_n = rowsq_parts(c);
+    a.rowsq_width = static_cast<float>(c.hidden);
+    a.eps = static_cast<float>(c.rms_eps);
     set_sk(a, sk);
     return cuda_check(launch_gemm_tc(Epi::kSwiGLU, a, st), "gate/up projection");
   }
@@ -315,11 +327,21 @@ int run_layer(const q3vl_config& c, const q3vl_layer& w, void* x, int64_t S, cha
   stage_event(3, st);
   Q3VL_TRY(run_attention(c, qkv, S, o, st));
   stage_event(4, st);
-  Q3VL_TRY(run_oproj(c, w, o, x, S, h, sk, st));
-  stage_event(5, st);
-  Q3VL_CUDA(launch_rowstat(c, h, S, c.hidden, inv2, st), "post-attention rms");
-  stage_event(6, st);
-  Q3VL_TRY(run_gateup(c, w, h, S, inv2, act, sk, st));
+  if (is_bf16(c)) {
+    // P7 fused: the o-projection epilogue leaves per-row sums of squares of
+    // h, which the gate/up epilogue turns into 1/rms
+    float* rowsq = reinterpret_cast<float*>(ws + L.rowsq);
+    Q3VL_TRY(run_oproj(c, w, o, x, S, h, sk, st, rowsq));
+    stage_event(5, st);
+    stage_event(6, st);
+    Q3VL_TRY(run_gateup(c, w, h, S, nullptr, act, sk, st, rowsq));
+  } else {
+    Q3VL_TRY(run_oproj(c, w, o, x, S, h, sk, st));
+    stage_event(5, st);
+    Q3VL_CUDA(launch_rowstat(c, h, S, c.hidden, inv2, st), "post-attention rms");
+    stage_event(6, st);
+    Q3VL_TRY(run_gateup(c, w, h, S, inv2, act, sk, st));
+  }
   stage_event(7, st);
   Q3VL_TRY(run_down(c, w, act, h, S, ds_slab, ds_slab ? map : nullptr, x, sk, st));
   stage_event(8, st);

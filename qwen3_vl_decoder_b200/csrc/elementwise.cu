@@ -234,11 +234,11 @@ __device__ __forceinline__ float sumsq16<__nv_bfloat16>(const uint4& v) {
   return s;
 }
 
-// Sum of squares of one row, read by a warp in batches of 8 16-byte vectors
+// Sum of squares of one row, read by a warp in batches of 16 16-byte vectors
 // per lane, all requested before any is used so the loads overlap.
 template <typename T>
 __device__ __forceinline__ float row_sumsq(const uint4* __restrict__ p, int64_t nvec, int lane) {
-  constexpr int kBatch = 8;
+  constexpr int kBatch = 16;
   float s = 0.f;
   for (int64_t base = 0; base < nvec; base += 32 * kBatch) {
     uint4 v[kBatch];

@@ -74,6 +74,11 @@ struct Params {
   // stream-K scratch: one fp32 128 x BN partial tile and one flag per CTA
   float* sk_partials;
   int32_t* sk_flags;
+  // row statistics between GEMMs (see GemmArgs)
+  float* rowsq_out;
+  const float* rowsq_in;
+  int rowsq_n;
+  float rowsq_width;
 };
 
 // Work schedule over 256 x BN pair tiles, shared by the roles of both CTAs of
@@ -165,6 +170,24 @@ __device__ __forceinline__ void stage_bf16x32(uint8_t* tile, int r, int cc, cons
     *reinterpret_cast<uint4*>(tile + out_off(r, cc, u)) =
         make_uint4(pack_bf16x2(v[8 * u + 0], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
                    pack_bf16x2(v[8 * u + 4], v[8 * u + 5]), pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
+}
+
+// stage_bf16x32 that also returns the sum of squares of the rounded values.
+__device__ __forceinline__ float stage_bf16x32_ss(uint8_t* tile, int r, int cc, const float* v) {
+  float ss = 0.f;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    uint32_t w[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const __nv_bfloat162 b = __floats2bfloat162_rn(v[8 * u + 2 * t], v[8 * u + 2 * t + 1]);
+      const float2 f = __bfloat1622float2(b);
+      ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+      w[t] = *reinterpret_cast<const uint32_t*>(&b);
+    }
+    *reinterpret_cast<uint4*>(tile + out_off(r, cc, u)) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  return ss;
 }
 
 __device__ __forceinline__ void add_staged_bf16x32(const uint8_t* tile, int r, int cc, float* v) {
@@ -506,7 +529,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             qkv_head<BN>(tbase + 128 * hh, 4 * hh, rr, part, n_part, slot_stride, row, valid,
                          n0 + 128 * hh, p, tile);
         } else if constexpr (EPI == static_cast<int>(Epi::kSwiGLU)) {
-          const float s = valid ? p.row_scale[row] : 0.f;
+          float s = 0.f;
+          if (valid) {
+            if (p.rowsq_in != nullptr) {
+              float ss = 0.f;
+              for (int t = 0; t < p.rowsq_n; ++t) ss += p.rowsq_in[row * p.rowsq_n + t];
+              s = 1.0f / sqrtf(ss / p.rowsq_width + p.eps);
+            } else {
+              s = p.row_scale[row];
+            }
+          }
 #pragma unroll 1
           for (int cc = 0; cc < 4; ++cc) {
             float g[32], u[32];
@@ -519,6 +551,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           }
         } else {
           const int32_t dsk = (kRes && valid && p.ds_map != nullptr) ? p.ds_map[row] : -1;
+          float ss = 0.f;
 #pragma unroll 1
           for (int cc = 0; cc < BN / 32; ++cc) {
             float v[32];
@@ -527,8 +560,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
               add_staged_bf16x32(tile, rr, cc, v);
               if (dsk >= 0) add_bf16x32(v, p.ds_slab + int64_t(dsk) * p.N + n0 + 32 * cc);
             }
-            stage_bf16x32(tile, rr, cc, v);
+            if (p.rowsq_out != nullptr) ss += stage_bf16x32_ss(tile, rr, cc, v);
+            else stage_bf16x32(tile, rr, cc, v);
           }
+          if (p.rowsq_out != nullptr && valid) p.rowsq_out[row * p.rowsq_n + tn] = ss;
         }
         fence_proxy_async_smem();
       }
@@ -654,6 +689,10 @@ cudaError_t launch_gemm_tc(Epi epi, const GemmArgs& a, cudaStream_t st) {
   p.err = device_error_ptr();
   p.sk_partials = a.sk_partials;
   p.sk_flags = a.sk_flags;
+  p.rowsq_out = a.rowsq_out;
+  p.rowsq_in = a.rowsq_in;
+  p.rowsq_n = a.rowsq_n;
+  p.rowsq_width = a.rowsq_width;
   if (a.K % BK != 0 || a.N % 128 != 0 || a.M <= 0) return cudaErrorInvalidValue;
   const bool use256 = a.N % 256 == 0;
   switch (epi) {
