@@ -374,6 +374,22 @@ def main():
     q3.check_device()
     assert torch.isfinite(st["out_host"].float()).all(), "non-finite output"
 
+    # a second workload for reference: the 2B-shape layer at S = 1024 (one GPU only)
+    also = {}
+    if world == 1 and args.workload != syn.Q2B_LAYER.name:
+        w2 = syn.Q2B_LAYER
+        st2 = setup(w2, dev)
+        for _ in range(5):
+            device_step(st2)
+        n2 = max(50, args.steps // 2)
+        t2 = timed(lambda k: device_step(st2), n2, world, dev)
+        st2["q3"].check_device()
+        g2, a2 = layer_flops(w2)
+        also[w2.name] = {"value": w2.seq * n2 / t2, "unit": UNIT, "ms_per_step": 1e3 * t2 / n2,
+                         "steps": n2, "tflops": (g2 + a2) * n2 / t2 / 1e12}
+        del st2
+        torch.cuda.empty_cache()
+
     burst, sustained, hbm, src = peaks()
     gemm_f, attn_f = layer_flops(w)
     H, I = w.hidden, w.intermediate
@@ -425,6 +441,7 @@ def main():
         "cpu_baseline": cpu,
         "e2e": {"value": world * S * args.steps / t_e2e, "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": st["out_host"].numel() * 2},
+        "also": also,
         "gpu_launches": launches,
         "clocks": clk.summary(),
         "next_position": nxt,

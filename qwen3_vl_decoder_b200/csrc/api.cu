@@ -69,6 +69,7 @@ WsLayout ws_layout(const q3vl_config& c, int64_t S) {
   L.act = take(size_t(S) * c.intermediate * e);
   if (c.dtype == Q3VL_DTYPE_BF16) {
     L.rowsq = take(size_t(S) * (c.hidden / 128) * sizeof(float));
+    L.rowsq_x = take(size_t(S) * (c.hidden / 128) * sizeof(float));
     L.sk_slots = sm_count();
     L.sk_part = take(size_t(L.sk_slots) * kSkSlotBytes);
     L.sk_flags = take(size_t(L.sk_slots) * sizeof(int32_t));
@@ -238,13 +239,19 @@ int clear_sk_flags(const Sk& k, cudaStream_t st) {
                     "clear stream-K flags");
 }
 
+int rowsq_parts(const q3vl_config& c);
+
 int run_qkv(const q3vl_config& c, const q3vl_layer& w, const void* x, int64_t S, const float* inv,
-            const float* cs, void* qkv, const Sk& sk, cudaStream_t st) {
+            const float* cs, void* qkv, const Sk& sk, cudaStream_t st,
+            const float* rowsq_in = nullptr) {
   GemmArgs a{};
   a.A = x; a.B = w.w_qkv; a.M = S; a.N = qkv_dim(c); a.K = c.hidden;
   a.out = qkv; a.ldo = a.N; a.row_scale = inv; a.bias = w.b_qkv;
   a.q_norm = w.q_norm; a.k_norm = w.k_norm; a.cos_sin = cs;
   a.q_cols = q_dim(c); a.k_cols = kv_dim(c); a.eps = static_cast<float>(c.rms_eps);
+  a.rowsq_in = rowsq_in;
+  a.rowsq_n = rowsq_parts(c);
+  a.rowsq_width = static_cast<float>(c.hidden);
   set_sk(a, sk);
   if (is_bf16(c)) return cuda_check(launch_gemm_tc(Epi::kQkv, a, st), "qkv projection");
   Q3VL_CUDA(launch_gemm_f32(Epi::kPlain, a, st), "qkv projection");
@@ -297,10 +304,13 @@ int run_gateup(const q3vl_config& c, const q3vl_layer& w, const void* h, int64_t
 }
 
 int run_down(const q3vl_config& c, const q3vl_layer& w, const void* act, const void* h, int64_t S,
-             const void* ds_slab, const int32_t* ds_map, void* out, const Sk& sk, cudaStream_t st) {
+             const void* ds_slab, const int32_t* ds_map, void* out, const Sk& sk, cudaStream_t st,
+             float* rowsq_out = nullptr) {
   GemmArgs a{};
   a.A = act; a.B = w.w_down; a.M = S; a.N = c.hidden; a.K = c.intermediate;
   a.out = out; a.ldo = c.hidden; a.resid = h;
+  a.rowsq_out = rowsq_out;
+  a.rowsq_n = rowsq_parts(c);
   a.ds_slab = ds_map ? ds_slab : nullptr;
   a.ds_map = ds_slab ? ds_map : nullptr;
   set_sk(a, sk);
@@ -310,8 +320,12 @@ int run_down(const q3vl_config& c, const q3vl_layer& w, const void* act, const v
 
 // The layer body on a prepared workspace (cos/sin table and DeepStack map
 // already written).
+// `x_stats_ready`: the previous layer of a stack left the row statistics of
+// x in the workspace, so P2 is skipped; `leave_x_stats`: this layer's down
+// epilogue leaves them for the next layer (bf16 path only).
 int run_layer(const q3vl_config& c, const q3vl_layer& w, void* x, int64_t S, char* ws,
-              const WsLayout& L, const void* ds_slab, cudaStream_t st) {
+              const WsLayout& L, const void* ds_slab, cudaStream_t st, bool x_stats_ready = false,
+              bool leave_x_stats = false) {
   float* cs = reinterpret_cast<float*>(ws + L.cos_sin);
   float* inv1 = reinterpret_cast<float*>(ws + L.inv1);
   float* inv2 = reinterpret_cast<float*>(ws + L.inv2);
@@ -321,9 +335,11 @@ int run_layer(const q3vl_config& c, const q3vl_layer& w, void* x, int64_t S, cha
   void* h = ws + L.h;
   void* act = ws + L.act;
   const Sk sk = sk_of(L, ws);
-  Q3VL_CUDA(launch_rowstat(c, x, S, c.hidden, inv1, st), "input rms");
+  float* rowsq_x = is_bf16(c) ? reinterpret_cast<float*>(ws + L.rowsq_x) : nullptr;
+  const bool use_x_stats = is_bf16(c) && x_stats_ready;
+  if (!use_x_stats) Q3VL_CUDA(launch_rowstat(c, x, S, c.hidden, inv1, st), "input rms");
   stage_event(2, st);
-  Q3VL_TRY(run_qkv(c, w, x, S, inv1, cs, qkv, sk, st));
+  Q3VL_TRY(run_qkv(c, w, x, S, inv1, cs, qkv, sk, st, use_x_stats ? rowsq_x : nullptr));
   stage_event(3, st);
   Q3VL_TRY(run_attention(c, qkv, S, o, st));
   stage_event(4, st);
@@ -343,7 +359,8 @@ int run_layer(const q3vl_config& c, const q3vl_layer& w, void* x, int64_t S, cha
     Q3VL_TRY(run_gateup(c, w, h, S, inv2, act, sk, st));
   }
   stage_event(7, st);
-  Q3VL_TRY(run_down(c, w, act, h, S, ds_slab, ds_slab ? map : nullptr, x, sk, st));
+  Q3VL_TRY(run_down(c, w, act, h, S, ds_slab, ds_slab ? map : nullptr, x, sk, st,
+                    is_bf16(c) && leave_x_stats ? rowsq_x : nullptr));
   stage_event(8, st);
   return Q3VL_OK;
 }
@@ -613,7 +630,8 @@ int q3vl_stack_prefill(const q3vl_config* cfg, int32_t n_layers, const q3vl_laye
   g_stage_events_on = false;  // stage events describe single-layer calls only
   for (int32_t l = 0; l < n_layers; ++l) {
     const void* slab = l < n_ds ? ds_slabs[l] : nullptr;
-    const int rc = run_layer(*cfg, layers[l], x, S, w, L, slab, st);
+    // P2 of layer l > 0 comes from layer l-1's down epilogue
+    const int rc = run_layer(*cfg, layers[l], x, S, w, L, slab, st, l > 0, l + 1 < n_layers);
     if (rc != Q3VL_OK) g_stage_events_on = events;
     if (rc != Q3VL_OK) return set_error(rc, "layer " + std::to_string(l) + ": " + g_last_error);
   }

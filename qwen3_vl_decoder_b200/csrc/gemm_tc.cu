@@ -264,7 +264,14 @@ __device__ __forceinline__ void qkv_head(uint32_t taddr, int cc0, int rr, const 
   for (int j = 0; j < 4; ++j)
     load_chunk<BN>(taddr + 32 * j, cc0 + j, rr, part, n_part, slot_stride, v + 32 * j);
   if (valid) {
-    const float s = p.row_scale[row];
+    float s;
+    if (p.rowsq_in != nullptr) {
+      float ss = 0.f;
+      for (int t = 0; t < p.rowsq_n; ++t) ss += p.rowsq_in[row * p.rowsq_n + t];
+      s = 1.0f / sqrtf(ss / p.rowsq_width + p.eps);
+    } else {
+      s = p.row_scale[row];
+    }
 #pragma unroll
     for (int t = 0; t < 128; ++t) v[t] *= s;
     if (p.bias != nullptr) {

@@ -34,7 +34,8 @@ struct WsLayout {
   size_t o = 0;        // dtype [S][Dq]
   size_t h = 0;        // dtype [S][H]
   size_t act = 0;      // dtype [S][I]
-  size_t rowsq = 0;    // fp32 [S][H/256] sums of squares of h per 256 columns (bf16 path)
+  size_t rowsq = 0;    // fp32 [S][H/128] sums of squares of h per N tile (bf16 path)
+  size_t rowsq_x = 0;  // fp32 [S][H/128] the same for x' (read by the next layer of a stack)
   size_t sk_part = 0;  // fp32 [sk_slots][128 x 256] stream-K partial tiles
   size_t sk_flags = 0; // int32 [sk_slots], zero between GEMM launches
   int sk_slots = 0;
@@ -103,8 +104,8 @@ struct GemmArgs {
   size_t sk_slot_bytes;
   // row statistics carried between GEMMs (bf16 tensor-core path):
   // kResidual may write, per row and per 256-column tile, the sum of squares
-  // of its bf16 output to rowsq_out[row * rowsq_n + tile]; kSwiGLU may read
-  // those rowsq_n partials instead of row_scale, as
+  // of its bf16 output to rowsq_out[row * rowsq_n + tile]; kSwiGLU and kQkv
+  // may read those rowsq_n partials instead of row_scale, as
   // 1 / sqrt(sum / rowsq_width + eps).
   float* rowsq_out;
   const float* rowsq_in;

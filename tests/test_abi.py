@@ -59,7 +59,7 @@ def test_sizes(lib):
     S = 4096
     ws = lib.q3vl_workspace_bytes(ctypes.byref(c), S)
     sk = 148 * (128 * 256 * 4 + 4)   # stream-K partial tiles and flags (148 SMs)
-    rowsq = S * (H // 128) * 4          # per-row sums of squares of h (P7 fused)
+    rowsq = 2 * S * (H // 128) * 4      # per-row sums of squares of h and x' (fused P7, P2)
     need = 2 * S * ((Dq + 2 * Dkv) + Dq + H + I) + S * (64 * 8 + 12) + sk + rowsq
     assert need <= ws <= need + 16 * 256
     assert lib.q3vl_workspace_bytes(ctypes.byref(c), 0) == 0

@@ -4,8 +4,10 @@ and the 32B-shape 50-layer prompt encoder, at full size.
 Per layer, teacher-forced: layer l's GPU output is compared with the oracle
 applied to the GPU's own layer-l input, on sampled rows (the oracle forms K/V
 for every row and the rest only for the sampled rows). The stack call must
-equal the layer-by-layer sequence bit for bit, and its final norm must match
-the oracle's.
+agree with the layer-by-layer sequence (it differs only in how the input row
+statistic of layers after the first is summed: from the previous layer's
+down epilogue instead of a separate pass), and its final norm must match the
+oracle's.
 """
 import numpy as np
 import pytest
@@ -71,7 +73,7 @@ def test_2b_stack28_deepstack_final_norm():
     xs = x0.clone()
     m.stack_prefill(cfg, packed, xs, pos, gain.cuda(), slabs_d, rows_d, ws)
     m.check_device()
-    assert torch.equal(xs, by_layer)
+    assert rel_l2(host(xs), host(by_layer)) <= 1e-2
     ref_norm = O.rms_norm(host(x), host(gain), w.rms_eps)
     assert rel_l2(host(xs), ref_norm) <= 1e-2
 
@@ -118,4 +120,4 @@ def test_32b_encoder50_no_final_norm(encoder32b, S):
         else:
             m.layer_prefill(cfg, packed[l], x, pos, None, None, ws)
     m.check_device()
-    assert torch.equal(x, xs)
+    assert rel_l2(host(xs), host(x)) <= 1e-2
