@@ -1,13 +1,13 @@
 """Layer stacks on the GPU: the 2B 28-layer stack with DeepStack and final norm,
 and the 32B-shape 50-layer prompt encoder, at full size.
 
-Per layer, teacher-forced: layer l's GPU output is compared with the oracle
-applied to the GPU's own layer-l input, on sampled rows (the oracle forms K/V
-for every row and the rest only for the sampled rows). The stack call must
-agree with the layer-by-layer sequence (it differs only in how the input row
-statistic of layers after the first is summed: from the previous layer's
-down epilogue instead of a separate pass), and its final norm must match the
-oracle's.
+The stack call itself is checked layer by layer, teacher-forced: running it
+on the first L layers gives x_L, and x_L must match the oracle's layer L-1
+applied to x_{L-1} (the same call on L-1 layers), on sampled rows (the oracle
+forms K/V for every row and the rest only for the sampled rows). Layers after
+the first take their input row statistic from the previous layer's down
+epilogue inside the stack, so this exercises that path. The final norm must
+match the oracle's norm of x_L.
 """
 import numpy as np
 import pytest
@@ -55,26 +55,20 @@ def test_2b_stack28_deepstack_final_norm():
     gain = syn.final_norm(w)
     x0 = syn.hidden_input(w).cuda()
     ws = m.workspace(cfg, w.seq)
-
-    # layer by layer, teacher-forced against the oracle
-    x = x0.clone()
     rows = _rows(w, 16, 0)
-    for l in range(w.n_layers):
-        x_in = x.clone()
-        slab = slabs_d[l] if l < len(slabs_d) else None
-        m.layer_prefill(cfg, packed[l], x, pos, slab, rows_d if slab is not None else None, ws)
+    prev = x0.clone()
+    for L in range(1, w.n_layers + 1):
+        x = x0.clone()
+        m.stack_prefill(cfg, packed[:L], x, pos, None, slabs_d, rows_d, ws)
         m.check_device()
-        _check_layer(w, raws[l], x_in.cpu(), x, pos_ref, rows,
+        l = L - 1
+        _check_layer(w, raws[l], prev.cpu(), x, pos_ref, rows,
                      slabs[l] if l < len(slabs) else None, ds_rows if l < len(slabs) else None)
-    by_layer = x.clone()
-    m.final_norm(cfg, by_layer, gain.cuda())
-
-    # the stack call is the same sequence
+        prev = x
     xs = x0.clone()
     m.stack_prefill(cfg, packed, xs, pos, gain.cuda(), slabs_d, rows_d, ws)
     m.check_device()
-    assert rel_l2(host(xs), host(by_layer)) <= 1e-2
-    ref_norm = O.rms_norm(host(x), host(gain), w.rms_eps)
+    ref_norm = O.rms_norm(host(prev), host(gain), w.rms_eps)
     assert rel_l2(host(xs), ref_norm) <= 1e-2
 
 
@@ -104,20 +98,14 @@ def test_32b_encoder50_no_final_norm(encoder32b, S):
     x0 = syn.hidden_input(w).cuda()
     ws = m.workspace(cfg, S)
     rows = _rows(w, 12, 1)
-    # full 50-layer stack, no final norm: the unnormalised residual stream
-    xs = x0.clone()
-    m.stack_prefill(cfg, packed, xs, pos, None, (), None, ws)
-    m.check_device()
-    assert torch.isfinite(xs.float()).all()
-    # teacher-forced checks of the first and the last layer
-    x = x0.clone()
-    for l in range(w.n_layers):
-        if l in (0, w.n_layers - 1):
-            x_in = x.clone()
-            m.layer_prefill(cfg, packed[l], x, pos, None, None, ws)
-            raw = {k: v.cpu() for k, v in syn.layer_weights(w, l, device="cuda").items()}
-            _check_layer(w, raw, x_in.cpu(), x, pos_ref, rows)
-        else:
-            m.layer_prefill(cfg, packed[l], x, pos, None, None, ws)
-    m.check_device()
-    assert rel_l2(host(xs), host(x)) <= 1e-2
+    xs = {}
+    for L in (1, w.n_layers - 1, w.n_layers):
+        x = x0.clone()
+        m.stack_prefill(cfg, packed[:L], x, pos, None, (), None, ws)
+        m.check_device()
+        assert torch.isfinite(x.float()).all()
+        xs[L] = x
+    xs[0] = x0
+    for l in (0, w.n_layers - 1):
+        raw = {k: v.cpu() for k, v in syn.layer_weights(w, l, device="cuda").items()}
+        _check_layer(w, raw, xs[l].cpu(), xs[l + 1], pos_ref, rows)
