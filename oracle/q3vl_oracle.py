@@ -19,15 +19,19 @@ Sources (the pages' own items; the pages print Rust, restated here):
 * inferencelayer ``vision.rs`` -- ``mrope_positions`` (token form: runs of
   image placeholders against a grid list, ``next`` position).
 * hf2q ``qwen3vl_text/forward.rs`` -- the module doc's per-layer order (bias
-  before the q/k norm), and the DeepStack contract and input validation of
-  ``forward_text_prefill_logits_last``.
+  before the q/k norm), the DeepStack contract and input validation of
+  ``forward_text_prefill_logits_last``, and "Why no KV cache yet" (a decoded
+  token is the last row of the prefill re-run over prompt + decoded tokens),
+  which defines the incremental decode at the end of this module.
 
 Parity status: every function here is pinned by the ``-m "not gpu"`` tests
 (hand-computed grids, closed forms, brute force, invariants). The composed
 random-weight layer is pinned through its parts and through closed-form
 special cases (zero projections, uniform attention, one-hot FFN); the pages
 print no numeric output of a full layer, so that composition has no external
-numeric pin.
+numeric pin. The decode functions are pinned against that prefill layer
+(the last row of a re-run prefill) and against closed forms that hold for
+arbitrary cache contents.
 """
 from __future__ import annotations
 
@@ -392,3 +396,108 @@ def stack(cfg: Config, layers: List[Dict], x, pos: np.ndarray, ds_slabs=(), ds_r
     if final_norm is not None:
         h = rms_norm(h, _np(final_norm, dtype), cfg.rms_eps)
     return h
+
+
+# ---------------------------------------------------------------------------
+# KV cache and incremental decode
+# ---------------------------------------------------------------------------
+#
+# hf2q ``qwen3vl_text/forward.rs``, module doc "Why no KV cache yet": the
+# first generation loop re-runs the whole prefill over prompt + tokens
+# decoded so far and keeps the last row; a KV cache only saves that work.
+# So a decoded token's output is, by definition, the last row of the prefill
+# over the extended sequence. The cache form below reaches the same numbers:
+# the K/V of the earlier rows do not depend on the new row (the layer is
+# causal), so they are computed once and kept.
+
+def text_positions_after(next_pos: int, n: int) -> np.ndarray:
+    """Positions of n text tokens that follow a prompt: all three axes equal
+    next_pos + i (inferencelayer ``vision.rs``: generation resumes one past
+    the largest position any axis reached, and a text token advances every
+    axis by one)."""
+    p = np.arange(next_pos, next_pos + n, dtype=np.int64)
+    return np.stack([p, p, p])
+
+
+def kv_rows(cfg: Config, W: Dict, x, pos: np.ndarray, dtype=np.float64):
+    """What a cache holds for rows 0..S-1 of one layer: K after the per-head
+    norm and MRoPE, and V, both [S, nkv, hd] (the k and v of ``qkv``)."""
+    x = _np(x, dtype)
+    angles = mrope_angles(pos, cfg.rope_theta, cfg.head_dim, cfg.mrope_section)
+    _, k, v = qkv(cfg, W, x, angles, dtype, q_rows=np.zeros(0, dtype=np.int64))
+    return k, v
+
+
+def layer_decode(cfg: Config, W: Dict, x_new, pos_new: np.ndarray, k_cache: Sequence,
+                 v_cache: Sequence, dtype=np.float64, taps: Optional[Dict] = None):
+    """One new token for each of B sequences through one layer.
+
+    x_new [B, H] are the new tokens' layer inputs, pos_new [3, B] their
+    positions, and k_cache[b] / v_cache[b] ([L_b, nkv, hd], L_b >= 0) the
+    cached K/V of sequence b's earlier rows. The new row attends to every
+    cached row and to itself (the causal row of the extended sequence).
+    Returns (x' [B, H], k_new [B, nkv, hd], v_new [B, nkv, hd]); k_new and
+    v_new are the rows a cache appends.
+    """
+    x_new = _np(x_new, dtype)
+    B = x_new.shape[0]
+    nh, nkv, hd = cfg.n_heads, cfg.n_kv_heads, cfg.head_dim
+    out = np.zeros_like(x_new)
+    k_new = np.zeros((B, nkv, hd), dtype=x_new.dtype)
+    v_new = np.zeros_like(k_new)
+    o_all = np.zeros((B, nh, hd), dtype=x_new.dtype)
+    for b in range(B):
+        angles = mrope_angles(np.asarray(pos_new)[:, b:b + 1], cfg.rope_theta, hd,
+                              cfg.mrope_section)
+        q, k, v = qkv(cfg, W, x_new[b:b + 1], angles, dtype)
+        kc = _np(k_cache[b], dtype).reshape(-1, nkv, hd)
+        vc = _np(v_cache[b], dtype).reshape(-1, nkv, hd)
+        L = kc.shape[0]
+        K = np.concatenate([kc, k], axis=0)
+        V = np.concatenate([vc, v], axis=0)
+        Q = np.zeros((L + 1, nh, hd), dtype=q.dtype)
+        Q[L] = q[0]
+        o = attention(Q, K, V, rows=np.array([L]))[L]
+        h = o_residual(W, o.reshape(1, nh * hd), x_new[b:b + 1], dtype)
+        a = ffn_act(cfg, W, h, dtype)
+        out[b] = down_residual(W, a, h, dtype)[0]
+        k_new[b], v_new[b], o_all[b] = k[0], v[0], o
+    if taps is not None:
+        taps.update(o=o_all, k=k_new, v=v_new)
+    return out, k_new, v_new
+
+
+def stack_prefill_kv(cfg: Config, layers: List[Dict], x, pos: np.ndarray, ds_slabs=(),
+                     ds_rows=None, final_norm=None, n_deepstack: int = 3, dtype=np.float64):
+    """``stack`` that also returns each layer's cache rows [(k, v), ...]:
+    layer l's K/V are formed from layer l's own input."""
+    h = _np(x, dtype)
+    if len(ds_slabs):
+        if len(ds_slabs) < n_deepstack:
+            raise OracleError("fewer DeepStack slabs than DeepStack layers")
+        if ds_rows is None or len(ds_rows) == 0:
+            raise OracleError("DeepStack slabs given without image rows")
+    caches = []
+    for li, W in enumerate(layers):
+        caches.append(kv_rows(cfg, W, h, pos, dtype))
+        slab = ds_slabs[li] if li < len(ds_slabs) else None
+        h = layer(cfg, W, h, pos, slab, ds_rows if slab is not None else None, dtype)
+    if final_norm is not None:
+        h = rms_norm(h, _np(final_norm, dtype), cfg.rms_eps)
+    return h, caches
+
+
+def stack_decode(cfg: Config, layers: List[Dict], x_new, pos_new: np.ndarray,
+                 caches: Sequence, final_norm=None, dtype=np.float64):
+    """One new token per sequence through every layer, then the optional final
+    norm. caches[l] = (k_cache, v_cache), each a per-sequence list as in
+    ``layer_decode``. Returns (y [B, H], [(k_new, v_new) per layer])."""
+    h = _np(x_new, dtype)
+    new = []
+    for li, W in enumerate(layers):
+        kc, vc = caches[li]
+        h, kn, vn = layer_decode(cfg, W, h, pos_new, kc, vc, dtype)
+        new.append((kn, vn))
+    if final_norm is not None:
+        h = rms_norm(h, _np(final_norm, dtype), cfg.rms_eps)
+    return h, new
