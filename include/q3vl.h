@@ -249,6 +249,78 @@ int q3vl_final_norm(const q3vl_config* cfg, void* x, int64_t S, const void* gain
                     q3vl_stream stream);
 
 /* ---------------------------------------------------------------------------
+ * KV cache and incremental decode (bf16 only; FP32 configs are refused with
+ * Q3VL_EUNSUPPORTED).
+ *
+ * [H] "Why no KV cache yet": a generation loop may re-run the prefill over
+ * prompt + tokens decoded so far and keep the last row; a KV cache gives the
+ * same result without re-running the earlier rows. The calls below keep,
+ * per layer, the K (after the per-head norm and MRoPE) and V rows of each
+ * sequence, and decode one new token per sequence against them.
+ * ------------------------------------------------------------------------- */
+
+/* One layer's cache (device memory owned by the caller). Row r of sequence
+ * slot s is at k + (s * cap + r) * nkv*hd elements (likewise v): K and V of
+ * every KV head of one token, head-major, exactly as the prefill's QKV step
+ * lays them out. */
+typedef struct q3vl_kv_cache {
+  void* k;        /* device bf16 [n_seq][cap][nkv*hd], 16-byte aligned */
+  void* v;        /* device bf16 [n_seq][cap][nkv*hd], 16-byte aligned */
+  int64_t cap;    /* rows per sequence slot, >= 1 */
+  int32_t n_seq;  /* sequence slots, >= 1 */
+} q3vl_kv_cache;
+
+/* q3vl_layer_prefill / q3vl_stack_prefill that also write rows 0..S-1 of
+ * sequence slot `seq` of each layer's cache (kv: host pointer to one cache
+ * for the layer call, to an array [n_layers] for the stack call). Requires
+ * S <= cap and 0 <= seq < n_seq (else Q3VL_ERANGE). Same workspace. */
+int q3vl_layer_prefill_kv(const q3vl_config* cfg, const q3vl_layer* layer, void* x, int64_t S,
+                          const int32_t* pos, const void* ds_slab, const int32_t* ds_rows,
+                          int32_t n_img, const q3vl_kv_cache* kv, int32_t seq, void* ws,
+                          size_t ws_bytes, q3vl_stream stream);
+int q3vl_stack_prefill_kv(const q3vl_config* cfg, int32_t n_layers, const q3vl_layer* layers,
+                          const void* final_norm, void* x, int64_t S, const int32_t* pos,
+                          const void* const* ds_slabs, int32_t n_ds, const int32_t* ds_rows,
+                          int32_t n_img, const q3vl_kv_cache* kv, int32_t seq, void* ws,
+                          size_t ws_bytes, q3vl_stream stream);
+
+/* Workspace bytes for the decode calls with batch B (1 <= B <= 256) against
+ * caches of `cap` rows per slot (0 for invalid arguments). */
+size_t q3vl_decode_workspace_bytes(const q3vl_config* cfg, int32_t B, int64_t cap);
+
+/* One new token for each of B sequences through one layer, in place:
+ * x[b] <- layer(x[b]) where token b attends to rows 0..len[b]-1 of cache
+ * slot seq[b] and to itself, and its own K/V row is written at row len[b]
+ * of that slot first (the same arithmetic as the prefill's row len[b]).
+ * x:   device bf16 [B, H] in/out, 16-byte aligned.
+ * pos: device int32 [3][B], the new tokens' (t, h, w) positions (a text
+ *      token after a prompt: next position + i on every axis).
+ * kv:  host pointer to this layer's cache.
+ * seq: device int32 [B], distinct slots in [0, n_seq).
+ * len: device int32 [B], rows already cached, 0 <= len[b] < cap. The call
+ *      reads but does not advance it (see q3vl_decode_advance).
+ * A seq or len out of range is recorded as the device error Q3VL_ERANGE and
+ * that token's output row is left unspecified.
+ * ws:  device workspace of >= q3vl_decode_workspace_bytes(cfg, B, cap)
+ *      bytes, 256-byte aligned. */
+int q3vl_layer_decode(const q3vl_config* cfg, const q3vl_layer* layer, void* x, int32_t B,
+                      const int32_t* pos, const q3vl_kv_cache* kv, const int32_t* seq,
+                      const int32_t* len, void* ws, size_t ws_bytes, q3vl_stream stream);
+
+/* n_layers layers of q3vl_layer_decode (kv: host array [n_layers]), then
+ * x <- RMSNorm(x, final_norm) when final_norm != NULL. The new tokens are
+ * text, so no DeepStack slab applies. */
+int q3vl_stack_decode(const q3vl_config* cfg, int32_t n_layers, const q3vl_layer* layers,
+                      const void* final_norm, void* x, int32_t B, const int32_t* pos,
+                      const q3vl_kv_cache* kv, const int32_t* seq, const int32_t* len, void* ws,
+                      size_t ws_bytes, q3vl_stream stream);
+
+/* After a decode step of text tokens: len[b] += 1 and pos[a][b] += 1 on all
+ * three axes (device int32 arrays [B] and [3][B]), so that a captured decode
+ * step can be replayed for the next token. */
+int q3vl_decode_advance(int32_t B, int32_t* pos, int32_t* len, q3vl_stream stream);
+
+/* ---------------------------------------------------------------------------
  * Diagnostics.
  * ------------------------------------------------------------------------- */
 

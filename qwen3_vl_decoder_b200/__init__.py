@@ -13,7 +13,7 @@ from typing import Dict, List, Optional, Sequence
 import torch
 
 from . import _abi
-from ._abi import Config, Layer, RawWeights  # noqa: F401
+from ._abi import Config, KvCache as KvCacheStruct, Layer, RawWeights  # noqa: F401
 
 _lib_handle: Optional[ctypes.CDLL] = None
 
@@ -156,7 +156,7 @@ def layer_prefill(cfg: Config, layer: PackedLayer, x: torch.Tensor, pos: torch.T
 def layer_prefill_noalloc(cfg: Config, layer: PackedLayer, x: torch.Tensor, pos: torch.Tensor,
                           ds_slab: Optional[torch.Tensor] = None,
                           ds_rows: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """layer_prefill with the library's built-in 32 MiB scratch instead of a workspace,
+    """layer_prefill with the library's built-in 64 MiB scratch instead of a workspace,
     for callers that cannot allocate device memory; calls must not overlap."""
     n_img = 0 if ds_rows is None else ds_rows.numel()
     _check(lib().q3vl_layer_prefill_noalloc(ctypes.byref(cfg), ctypes.byref(layer.views), _ptr(x),
@@ -179,6 +179,109 @@ def stack_prefill(cfg: Config, layers: Sequence[PackedLayer], x: torch.Tensor, p
                                    S, _ptr(pos), slabs if ds_slabs else None, len(ds_slabs),
                                    _ptr(ds_rows), n_img, _ptr(ws), ws.numel(), _stream(stream)))
     return x
+
+
+# ---------------------------------------------------------------------------
+# KV cache and one-token decode (bf16)
+# ---------------------------------------------------------------------------
+class KvCache:
+    """One layer's cache: k and v bf16 [n_seq, cap, nkv*128] on the device (K after the
+    per-head norm and MRoPE, as the prefill forms it)."""
+
+    def __init__(self, cfg: Config, n_seq: int, cap: int, device="cuda"):
+        dkv = cfg.n_kv_heads * cfg.head_dim
+        self.k = torch.zeros((n_seq, cap, dkv), dtype=torch.bfloat16, device=device)
+        self.v = torch.zeros_like(self.k)
+        self.struct = KvCacheStruct(self.k.data_ptr(), self.v.data_ptr(), cap, n_seq)
+
+    @property
+    def cap(self) -> int:
+        return int(self.struct.cap)
+
+
+def kv_caches(cfg: Config, n_layers: int, n_seq: int, cap: int, device="cuda") -> List[KvCache]:
+    return [KvCache(cfg, n_seq, cap, device) for _ in range(n_layers)]
+
+
+def _kv_array(kvs: Sequence[KvCache]):
+    return (KvCacheStruct * len(kvs))(*[kv.struct for kv in kvs])
+
+
+def layer_prefill_kv(cfg: Config, layer: PackedLayer, x: torch.Tensor, pos: torch.Tensor,
+                     kv: KvCache, seq: int = 0, ds_slab: Optional[torch.Tensor] = None,
+                     ds_rows: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """layer_prefill that also writes rows 0..S-1 of cache slot `seq`."""
+    S = x.shape[0]
+    ws = workspace(cfg, S, x.device) if ws is None else ws
+    n_img = 0 if ds_rows is None else ds_rows.numel()
+    _check(lib().q3vl_layer_prefill_kv(ctypes.byref(cfg), ctypes.byref(layer.views), _ptr(x), S,
+                                      _ptr(pos), _ptr(ds_slab), _ptr(ds_rows), n_img,
+                                      ctypes.byref(kv.struct), seq, _ptr(ws), ws.numel(),
+                                      _stream(stream)))
+    return x
+
+
+def stack_prefill_kv(cfg: Config, layers: Sequence[PackedLayer], x: torch.Tensor,
+                     pos: torch.Tensor, kvs: Sequence[KvCache], seq: int = 0,
+                     final_norm: Optional[torch.Tensor] = None,
+                     ds_slabs: Sequence[torch.Tensor] = (), ds_rows: Optional[torch.Tensor] = None,
+                     ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """stack_prefill that also writes each layer's rows 0..S-1 of cache slot `seq`."""
+    S = x.shape[0]
+    ws = workspace(cfg, S, x.device) if ws is None else ws
+    arr = (Layer * len(layers))(*[l.views for l in layers])
+    slabs = (ctypes.c_void_p * max(1, len(ds_slabs)))(*[s.data_ptr() for s in ds_slabs])
+    n_img = 0 if ds_rows is None else ds_rows.numel()
+    _check(lib().q3vl_stack_prefill_kv(ctypes.byref(cfg), len(layers), arr, _ptr(final_norm),
+                                      _ptr(x), S, _ptr(pos), slabs if ds_slabs else None,
+                                      len(ds_slabs), _ptr(ds_rows), n_img, _kv_array(kvs), seq,
+                                      _ptr(ws), ws.numel(), _stream(stream)))
+    return x
+
+
+def decode_workspace_bytes(cfg: Config, B: int, cap: int) -> int:
+    return int(lib().q3vl_decode_workspace_bytes(ctypes.byref(cfg), B, cap))
+
+
+def decode_workspace(cfg: Config, B: int, cap: int, device="cuda") -> torch.Tensor:
+    n = decode_workspace_bytes(cfg, B, cap)
+    if n == 0:
+        _check(_abi.EINVAL)
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def layer_decode(cfg: Config, layer: PackedLayer, x: torch.Tensor, pos: torch.Tensor,
+                 kv: KvCache, seq: torch.Tensor, lens: torch.Tensor,
+                 ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One new token per sequence (x [B, H] in place): token b's K/V go to row lens[b] of
+    slot seq[b], and it attends to rows 0..lens[b] of that slot."""
+    B = x.shape[0]
+    ws = decode_workspace(cfg, B, kv.cap, x.device) if ws is None else ws
+    _check(lib().q3vl_layer_decode(ctypes.byref(cfg), ctypes.byref(layer.views), _ptr(x), B,
+                                  _ptr(pos), ctypes.byref(kv.struct), _ptr(seq), _ptr(lens),
+                                  _ptr(ws), ws.numel(), _stream(stream)))
+    return x
+
+
+def stack_decode(cfg: Config, layers: Sequence[PackedLayer], x: torch.Tensor, pos: torch.Tensor,
+                 kvs: Sequence[KvCache], seq: torch.Tensor, lens: torch.Tensor,
+                 final_norm: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+    """layer_decode through every layer, then the optional final norm; x in place."""
+    B = x.shape[0]
+    cap = max(kv.cap for kv in kvs)
+    ws = decode_workspace(cfg, B, cap, x.device) if ws is None else ws
+    arr = (Layer * len(layers))(*[l.views for l in layers])
+    _check(lib().q3vl_stack_decode(ctypes.byref(cfg), len(layers), arr, _ptr(final_norm), _ptr(x),
+                                  B, _ptr(pos), _kv_array(kvs), _ptr(seq), _ptr(lens), _ptr(ws),
+                                  ws.numel(), _stream(stream)))
+    return x
+
+
+def decode_advance(pos: torch.Tensor, lens: torch.Tensor, stream=None) -> None:
+    """lens += 1 and every position axis += 1 (the next text token), on the device."""
+    _check(lib().q3vl_decode_advance(lens.numel(), _ptr(pos), _ptr(lens), _stream(stream)))
 
 
 # ---------------------------------------------------------------------------

@@ -38,6 +38,11 @@ class Layer(ctypes.Structure):
         "w_qkv", "b_qkv", "q_norm", "k_norm", "w_o", "w_gu", "w_down")]
 
 
+class KvCache(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("cap", ctypes.c_int64),
+                ("n_seq", ctypes.c_int32)]
+
+
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
 _I32 = ctypes.c_int32
@@ -69,6 +74,17 @@ SIGNATURES = {
                                  _P]),
     "q3vl_deepstack_map": (ctypes.c_int, [_P, _I32, _I64, _P, _P]),
     "q3vl_final_norm": (ctypes.c_int, [_CFG, _P, _I64, _P, _P]),
+    "q3vl_layer_prefill_kv": (ctypes.c_int, [_CFG, ctypes.POINTER(Layer), _P, _I64, _P, _P, _P,
+                                             _I32, ctypes.POINTER(KvCache), _I32, _P, _SZ, _P]),
+    "q3vl_stack_prefill_kv": (ctypes.c_int, [_CFG, _I32, ctypes.POINTER(Layer), _P, _P, _I64, _P,
+                                             ctypes.POINTER(_P), _I32, _P, _I32,
+                                             ctypes.POINTER(KvCache), _I32, _P, _SZ, _P]),
+    "q3vl_decode_workspace_bytes": (_SZ, [_CFG, _I32, _I64]),
+    "q3vl_layer_decode": (ctypes.c_int, [_CFG, ctypes.POINTER(Layer), _P, _I32, _P,
+                                         ctypes.POINTER(KvCache), _P, _P, _P, _SZ, _P]),
+    "q3vl_stack_decode": (ctypes.c_int, [_CFG, _I32, ctypes.POINTER(Layer), _P, _P, _I32, _P,
+                                         ctypes.POINTER(KvCache), _P, _P, _P, _SZ, _P]),
+    "q3vl_decode_advance": (ctypes.c_int, [_I32, _P, _P, _P]),
     "q3vl_device_status": (ctypes.c_int, [_P, ctypes.POINTER(_I32), ctypes.POINTER(_I32)]),
     "q3vl_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_uint32, _P]),
     "q3vl_set_stage_events": (ctypes.c_int, [ctypes.POINTER(_P), _I32]),

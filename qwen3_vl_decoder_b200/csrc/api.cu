@@ -323,9 +323,12 @@ int run_down(const q3vl_config& c, const q3vl_layer& w, const void* act, const v
 // `x_stats_ready`: the previous layer of a stack left the row statistics of
 // x in the workspace, so P2 is skipped; `leave_x_stats`: this layer's down
 // epilogue leaves them for the next layer (bf16 path only).
+// `kv` (optional): the K/V rows of this layer are also written into rows
+// 0..S-1 of slot `kv_seq` of that cache.
 int run_layer(const q3vl_config& c, const q3vl_layer& w, void* x, int64_t S, char* ws,
               const WsLayout& L, const void* ds_slab, cudaStream_t st, bool x_stats_ready = false,
-              bool leave_x_stats = false) {
+              bool leave_x_stats = false, const q3vl_kv_cache* kv = nullptr,
+              int32_t kv_seq = 0) {
   float* cs = reinterpret_cast<float*>(ws + L.cos_sin);
   float* inv1 = reinterpret_cast<float*>(ws + L.inv1);
   float* inv2 = reinterpret_cast<float*>(ws + L.inv2);
@@ -340,6 +343,7 @@ int run_layer(const q3vl_config& c, const q3vl_layer& w, void* x, int64_t S, cha
   if (!use_x_stats) Q3VL_CUDA(launch_rowstat(c, x, S, c.hidden, inv1, st), "input rms");
   stage_event(2, st);
   Q3VL_TRY(run_qkv(c, w, x, S, inv1, cs, qkv, sk, st, use_x_stats ? rowsq_x : nullptr));
+  if (kv != nullptr) Q3VL_CUDA(launch_kv_store(c, qkv, S, *kv, kv_seq, st), "kv cache store");
   stage_event(3, st);
   Q3VL_TRY(run_attention(c, qkv, S, o, st));
   stage_event(4, st);
@@ -388,6 +392,110 @@ int step_sk(const q3vl_config& c, int64_t S, void* ws, size_t ws_bytes, cudaStre
   Q3VL_TRY(check_ws(c, S, ws, ws_bytes));
   *out = sk_of(ws_layout(c, S), static_cast<char*>(ws));
   return clear_sk_flags(*out, st);
+}
+
+int check_kv(const q3vl_config& c, const q3vl_kv_cache* kv, const char* what) {
+  if (kv == nullptr) return set_error(Q3VL_EINVAL, std::string(what) + " is NULL");
+  Q3VL_TRY(check_ptr(kv->k, "kv cache k"));
+  Q3VL_TRY(check_ptr(kv->v, "kv cache v"));
+  if (kv->cap < 1 || kv->n_seq < 1)
+    return set_error(Q3VL_EINVAL, "kv cache needs cap >= 1 and n_seq >= 1");
+  (void)c;
+  return Q3VL_OK;
+}
+
+// The decode path covers bf16 layers whose query-group size is 1, 2, 4 or 8
+// and whose hidden size is a multiple of 128 (its projection row tiles).
+int check_decode_cfg(const q3vl_config& c) {
+  if (c.dtype != Q3VL_DTYPE_BF16)
+    return set_error(Q3VL_EUNSUPPORTED, "the KV cache and decode calls are bf16 only");
+  const int G = c.n_heads / c.n_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8)
+    return set_error(Q3VL_EUNSUPPORTED, "decode needs n_heads / n_kv_heads in {1, 2, 4, 8}");
+  if (c.hidden % 128 != 0)
+    return set_error(Q3VL_EUNSUPPORTED, "decode needs hidden to be a multiple of 128");
+  return Q3VL_OK;
+}
+
+int check_batch(int32_t B) {
+  if (B < 1 || B > 256) return set_error(Q3VL_EINVAL, "decode batch B must be in [1, 256]");
+  return Q3VL_OK;
+}
+
+int check_dec_ws(const q3vl_config& c, int32_t B, int64_t cap, const void* ws, size_t ws_bytes) {
+  const size_t need = dec_layout(c, B, cap).total;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255) != 0)
+    return set_error(Q3VL_EWORKSPACE, "workspace must be non-NULL and 256-byte aligned");
+  if (ws_bytes < need)
+    return set_error(Q3VL_EWORKSPACE, "decode workspace too small: need " + std::to_string(need) +
+                                          " bytes, got " + std::to_string(ws_bytes));
+  return Q3VL_OK;
+}
+
+// One layer of the decode on a prepared workspace (cos/sin of the B new
+// positions written, tickets zero). `x_stats_ready`: the previous layer's
+// down epilogue left the row sums of squares of x.
+int run_decode_layer(const q3vl_config& c, const q3vl_layer& w, void* x, int32_t B,
+                     const q3vl_kv_cache& kv, const int32_t* seq, const int32_t* len, char* ws,
+                     const DecLayout& L, cudaStream_t st, bool x_stats_ready, bool leave_x_stats) {
+  const int64_t H = c.hidden, I = c.intermediate, Dq = q_dim(c);
+  float* inv = reinterpret_cast<float*>(ws + L.inv);
+  float* rowsq_h = reinterpret_cast<float*>(ws + L.rowsq_h);
+  float* rowsq_x = reinterpret_cast<float*>(ws + L.rowsq_x);
+  float* part = reinterpret_cast<float*>(ws + L.part);
+  uint32_t* tickets = reinterpret_cast<uint32_t*>(ws + L.tickets);
+  void* q = ws + L.q;
+  void* o = ws + L.o;
+  void* h = ws + L.h;
+  void* act = ws + L.act;
+  if (!x_stats_ready) Q3VL_CUDA(launch_rowstat(c, x, B, H, inv, st), "decode input rms");
+
+  DecGemmArgs a{};
+  a.B = B; a.part = part; a.tickets = tickets; a.eps = static_cast<float>(c.rms_eps);
+  a.n_heads = c.n_heads; a.n_kv = c.n_kv_heads;
+  // P3+P4, with this token's K/V row written into the cache
+  a.W = w.w_qkv; a.rows = qkv_dim(c); a.K = H; a.X = x;
+  a.N = Dq; a.out = q; a.inv = inv;
+  a.rowsq_in = x_stats_ready ? rowsq_x : nullptr;
+  a.rowsq_n = static_cast<int>(H / 128); a.rowsq_width = static_cast<float>(H);
+  a.bias = w.b_qkv; a.q_norm = w.q_norm; a.k_norm = w.k_norm;
+  a.cos_sin = reinterpret_cast<const float*>(ws + L.cos_sin);
+  a.k_cache = kv.k; a.v_cache = kv.v; a.cap = kv.cap; a.n_seq = kv.n_seq; a.seq = seq; a.len = len;
+  Q3VL_CUDA(launch_decode_gemm(Epi::kQkv, a, st), "decode qkv projection");
+  // P5 over the cache
+  Q3VL_CUDA(launch_decode_attention(c, q, kv, seq, len, B, o,
+                                    reinterpret_cast<float*>(ws + L.att_part),
+                                    reinterpret_cast<uint32_t*>(ws + L.att_tickets), L.att_items,
+                                    st),
+            "decode attention");
+  // P6 (+ the row sums of squares of h for P7)
+  DecGemmArgs r{};
+  r.B = B; r.part = part; r.tickets = tickets; r.eps = a.eps;
+  r.W = w.w_o; r.rows = H; r.K = Dq; r.X = o;
+  r.N = H; r.out = h; r.resid = x; r.rowsq_out = rowsq_h;
+  Q3VL_CUDA(launch_decode_gemm(Epi::kResidual, r, st), "decode o projection");
+  // P7+P8
+  DecGemmArgs g{};
+  g.B = B; g.part = part; g.tickets = tickets; g.eps = a.eps;
+  g.W = w.w_gu; g.rows = 2 * I; g.K = H; g.X = h;
+  g.N = I; g.out = act; g.rowsq_in = rowsq_h;
+  g.rowsq_n = static_cast<int>(H / 128); g.rowsq_width = static_cast<float>(H);
+  Q3VL_CUDA(launch_decode_gemm(Epi::kSwiGLU, g, st), "decode gate/up projection");
+  // P9 (+ the row sums of squares of x' for the next layer)
+  DecGemmArgs d{};
+  d.B = B; d.part = part; d.tickets = tickets; d.eps = a.eps;
+  d.W = w.w_down; d.rows = H; d.K = I; d.X = act;
+  d.N = H; d.out = x; d.resid = h; d.rowsq_out = leave_x_stats ? rowsq_x : nullptr;
+  Q3VL_CUDA(launch_decode_gemm(Epi::kResidual, d, st), "decode down projection");
+  return Q3VL_OK;
+}
+
+// Positions' cos/sin and zero tickets: once per decode call.
+int prepare_decode(const q3vl_config& c, const int32_t* pos, int32_t B, char* ws,
+                   const DecLayout& L, cudaStream_t st) {
+  Q3VL_CUDA(cudaMemsetAsync(ws + L.tickets, 0, L.total - L.tickets, st), "clear decode tickets");
+  return cuda_check(launch_rope_table(c, pos, B, reinterpret_cast<float*>(ws + L.cos_sin), st),
+                    "decode rope table");
 }
 
 }  // namespace
@@ -561,9 +669,10 @@ int q3vl_final_norm(const q3vl_config* cfg, void* x, int64_t S, const void* gain
   return cuda_check(launch_final_norm(*cfg, x, S, gain, ST(stream)), "final norm");
 }
 
-int q3vl_layer_prefill(const q3vl_config* cfg, const q3vl_layer* layer, void* x, int64_t S,
-                       const int32_t* pos, const void* ds_slab, const int32_t* ds_rows,
-                       int32_t n_img, void* ws, size_t ws_bytes, q3vl_stream stream) {
+static int layer_prefill_impl(const q3vl_config* cfg, const q3vl_layer* layer, void* x, int64_t S,
+                              const int32_t* pos, const void* ds_slab, const int32_t* ds_rows,
+                              int32_t n_img, const q3vl_kv_cache* kv, int32_t kv_seq, void* ws,
+                              size_t ws_bytes, q3vl_stream stream) {
   Q3VL_TRY(check_cfg(cfg));
   Q3VL_TRY(check_seq(S));
   Q3VL_TRY(check_layer(cfg, layer));
@@ -587,13 +696,45 @@ int q3vl_layer_prefill(const q3vl_config* cfg, const q3vl_layer* layer, void* x,
     Q3VL_CUDA(launch_deepstack_map(ds_rows, n_img, S, reinterpret_cast<int32_t*>(w + L.ds_map), st),
               "deepstack map");
   stage_event(1, st);
-  return run_layer(*cfg, *layer, x, S, w, L, ds_slab, st);
+  return run_layer(*cfg, *layer, x, S, w, L, ds_slab, st, false, false, kv, kv_seq);
 }
 
-int q3vl_stack_prefill(const q3vl_config* cfg, int32_t n_layers, const q3vl_layer* layers,
-                       const void* final_norm, void* x, int64_t S, const int32_t* pos,
-                       const void* const* ds_slabs, int32_t n_ds, const int32_t* ds_rows,
+// Cache checks of the *_kv prefill calls: bf16, rows 0..S-1 of one slot.
+static int check_prefill_kv(const q3vl_config* cfg, int64_t S, const q3vl_kv_cache* kv,
+                            int32_t n, int32_t seq) {
+  Q3VL_TRY(check_cfg(cfg));
+  if (cfg->dtype != Q3VL_DTYPE_BF16)
+    return set_error(Q3VL_EUNSUPPORTED, "the KV cache and decode calls are bf16 only");
+  if (kv == nullptr) return set_error(Q3VL_EINVAL, "kv is NULL");
+  for (int32_t l = 0; l < n; ++l) {
+    Q3VL_TRY(check_kv(*cfg, kv + l, "kv"));
+    if (S > kv[l].cap) return set_error(Q3VL_ERANGE, "S exceeds the cache capacity");
+    if (seq < 0 || seq >= kv[l].n_seq) return set_error(Q3VL_ERANGE, "seq outside [0, n_seq)");
+  }
+  return Q3VL_OK;
+}
+
+int q3vl_layer_prefill(const q3vl_config* cfg, const q3vl_layer* layer, void* x, int64_t S,
+                       const int32_t* pos, const void* ds_slab, const int32_t* ds_rows,
                        int32_t n_img, void* ws, size_t ws_bytes, q3vl_stream stream) {
+  return layer_prefill_impl(cfg, layer, x, S, pos, ds_slab, ds_rows, n_img, nullptr, 0, ws,
+                            ws_bytes, stream);
+}
+
+int q3vl_layer_prefill_kv(const q3vl_config* cfg, const q3vl_layer* layer, void* x, int64_t S,
+                          const int32_t* pos, const void* ds_slab, const int32_t* ds_rows,
+                          int32_t n_img, const q3vl_kv_cache* kv, int32_t seq, void* ws,
+                          size_t ws_bytes, q3vl_stream stream) {
+  Q3VL_TRY(check_prefill_kv(cfg, S, kv, 1, seq));
+  return layer_prefill_impl(cfg, layer, x, S, pos, ds_slab, ds_rows, n_img, kv, seq, ws,
+                            ws_bytes, stream);
+}
+
+static int stack_prefill_impl(const q3vl_config* cfg, int32_t n_layers, const q3vl_layer* layers,
+                              const void* final_norm, void* x, int64_t S, const int32_t* pos,
+                              const void* const* ds_slabs, int32_t n_ds, const int32_t* ds_rows,
+                              int32_t n_img, const q3vl_kv_cache* kv, int32_t kv_seq, void* ws,
+                              size_t ws_bytes, q3vl_stream stream) {
   Q3VL_TRY(check_cfg(cfg));
   Q3VL_TRY(check_seq(S));
   if (n_layers <= 0 || layers == nullptr)
@@ -631,7 +772,8 @@ int q3vl_stack_prefill(const q3vl_config* cfg, int32_t n_layers, const q3vl_laye
   for (int32_t l = 0; l < n_layers; ++l) {
     const void* slab = l < n_ds ? ds_slabs[l] : nullptr;
     // P2 of layer l > 0 comes from layer l-1's down epilogue
-    const int rc = run_layer(*cfg, layers[l], x, S, w, L, slab, st, l > 0, l + 1 < n_layers);
+    const int rc = run_layer(*cfg, layers[l], x, S, w, L, slab, st, l > 0, l + 1 < n_layers,
+                             kv != nullptr ? kv + l : nullptr, kv_seq);
     if (rc != Q3VL_OK) g_stage_events_on = events;
     if (rc != Q3VL_OK) return set_error(rc, "layer " + std::to_string(l) + ": " + g_last_error);
   }
@@ -639,6 +781,94 @@ int q3vl_stack_prefill(const q3vl_config* cfg, int32_t n_layers, const q3vl_laye
   if (final_norm != nullptr)
     Q3VL_CUDA(launch_final_norm(*cfg, x, S, final_norm, st), "final norm");
   return Q3VL_OK;
+}
+
+int q3vl_stack_prefill(const q3vl_config* cfg, int32_t n_layers, const q3vl_layer* layers,
+                       const void* final_norm, void* x, int64_t S, const int32_t* pos,
+                       const void* const* ds_slabs, int32_t n_ds, const int32_t* ds_rows,
+                       int32_t n_img, void* ws, size_t ws_bytes, q3vl_stream stream) {
+  return stack_prefill_impl(cfg, n_layers, layers, final_norm, x, S, pos, ds_slabs, n_ds,
+                            ds_rows, n_img, nullptr, 0, ws, ws_bytes, stream);
+}
+
+int q3vl_stack_prefill_kv(const q3vl_config* cfg, int32_t n_layers, const q3vl_layer* layers,
+                          const void* final_norm, void* x, int64_t S, const int32_t* pos,
+                          const void* const* ds_slabs, int32_t n_ds, const int32_t* ds_rows,
+                          int32_t n_img, const q3vl_kv_cache* kv, int32_t seq, void* ws,
+                          size_t ws_bytes, q3vl_stream stream) {
+  if (n_layers <= 0) return set_error(Q3VL_EINVAL, "n_layers must be >= 1");
+  Q3VL_TRY(check_prefill_kv(cfg, S, kv, n_layers, seq));
+  return stack_prefill_impl(cfg, n_layers, layers, final_norm, x, S, pos, ds_slabs, n_ds,
+                            ds_rows, n_img, kv, seq, ws, ws_bytes, stream);
+}
+
+size_t q3vl_decode_workspace_bytes(const q3vl_config* cfg, int32_t B, int64_t cap) {
+  if (check_cfg(cfg) != Q3VL_OK || check_decode_cfg(*cfg) != Q3VL_OK || check_batch(B) != Q3VL_OK ||
+      cap < 1)
+    return 0;
+  return dec_layout(*cfg, B, cap).total;
+}
+
+static int decode_checks(const q3vl_config* cfg, int32_t n_layers, const q3vl_layer* layers,
+                         void* x, int32_t B, const int32_t* pos, const q3vl_kv_cache* kv,
+                         const int32_t* seq, const int32_t* len, void* ws, size_t ws_bytes) {
+  Q3VL_TRY(check_cfg(cfg));
+  Q3VL_TRY(check_decode_cfg(*cfg));
+  Q3VL_TRY(check_batch(B));
+  if (layers == nullptr || kv == nullptr) return set_error(Q3VL_EINVAL, "layers / kv are NULL");
+  int64_t cap = 0;
+  for (int32_t l = 0; l < n_layers; ++l) {
+    const int rc = check_layer(cfg, layers + l);
+    if (rc != Q3VL_OK) return set_error(rc, "layer " + std::to_string(l) + ": " + g_last_error);
+    Q3VL_TRY(check_kv(*cfg, kv + l, "kv"));
+    if (kv[l].cap > cap) cap = kv[l].cap;
+  }
+  Q3VL_TRY(check_ptr(x, "x"));
+  Q3VL_TRY(check_ptr(pos, "pos", false));
+  Q3VL_TRY(check_ptr(seq, "seq", false));
+  Q3VL_TRY(check_ptr(len, "len", false));
+  return check_dec_ws(*cfg, B, cap, ws, ws_bytes);
+}
+
+int q3vl_layer_decode(const q3vl_config* cfg, const q3vl_layer* layer, void* x, int32_t B,
+                      const int32_t* pos, const q3vl_kv_cache* kv, const int32_t* seq,
+                      const int32_t* len, void* ws, size_t ws_bytes, q3vl_stream stream) {
+  Q3VL_TRY(decode_checks(cfg, 1, layer, x, B, pos, kv, seq, len, ws, ws_bytes));
+  const cudaStream_t st = ST(stream);
+  const DecLayout L = dec_layout(*cfg, B, kv->cap);
+  char* w = static_cast<char*>(ws);
+  Q3VL_TRY(prepare_decode(*cfg, pos, B, w, L, st));
+  return run_decode_layer(*cfg, *layer, x, B, *kv, seq, len, w, L, st, false, false);
+}
+
+int q3vl_stack_decode(const q3vl_config* cfg, int32_t n_layers, const q3vl_layer* layers,
+                      const void* final_norm, void* x, int32_t B, const int32_t* pos,
+                      const q3vl_kv_cache* kv, const int32_t* seq, const int32_t* len, void* ws,
+                      size_t ws_bytes, q3vl_stream stream) {
+  if (n_layers <= 0) return set_error(Q3VL_EINVAL, "n_layers must be >= 1");
+  Q3VL_TRY(decode_checks(cfg, n_layers, layers, x, B, pos, kv, seq, len, ws, ws_bytes));
+  if (final_norm != nullptr) Q3VL_TRY(check_ptr(final_norm, "final_norm"));
+  int64_t cap = 0;
+  for (int32_t l = 0; l < n_layers; ++l) cap = kv[l].cap > cap ? kv[l].cap : cap;
+  const cudaStream_t st = ST(stream);
+  const DecLayout L = dec_layout(*cfg, B, cap);
+  char* w = static_cast<char*>(ws);
+  Q3VL_TRY(prepare_decode(*cfg, pos, B, w, L, st));
+  for (int32_t l = 0; l < n_layers; ++l) {
+    const int rc = run_decode_layer(*cfg, layers[l], x, B, kv[l], seq, len, w, L, st, l > 0,
+                                    l + 1 < n_layers);
+    if (rc != Q3VL_OK) return set_error(rc, "layer " + std::to_string(l) + ": " + g_last_error);
+  }
+  if (final_norm != nullptr)
+    Q3VL_CUDA(launch_final_norm(*cfg, x, B, final_norm, st), "final norm");
+  return Q3VL_OK;
+}
+
+int q3vl_decode_advance(int32_t B, int32_t* pos, int32_t* len, q3vl_stream stream) {
+  Q3VL_TRY(check_batch(B));
+  Q3VL_TRY(check_ptr(pos, "pos", false));
+  Q3VL_TRY(check_ptr(len, "len", false));
+  return cuda_check(launch_decode_advance(B, pos, len, ST(stream)), "decode advance");
 }
 
 int q3vl_set_stage_events(void* const* events, int32_t n_events) {

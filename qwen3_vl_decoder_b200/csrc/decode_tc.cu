@@ -1,0 +1,771 @@
+// One-token-per-sequence decode on sm_100a: the KV cache writes of the
+// prefill, the skinny projections (tcgen05, swap-AB, split-K), the
+// split-sequence attention over the cache, and the step that advances
+// positions and lengths.
+//
+// Why a decoded token needs no re-run of the prompt: hf2q
+// qwen3vl_text/forward.rs, module doc "Why no KV cache yet" (the generation
+// loop may re-run the prefill over prompt + decoded tokens and keep the last
+// row; the cache keeps the earlier rows' K/V instead). The per-token
+// arithmetic is the prefill's (cortiq-engine qwen3te.rs,
+// `Qwen3Encoder::encode_with_images` loop body; `Qwen3Encoder::norm_rope`;
+// `rms_norm_into`; `silu`).
+//
+// Projections. With B <= 256 tokens the layer streams each weight matrix
+// once, so the work is bound by HBM, not by the tensor cores. The weight
+// matrix is the MMA's M operand (128 rows per tile, or 256 for gate/up whose
+// packed rows interleave 128 gate and 128 up rows) and the tokens are its N
+// operand (B rounded up to 16; TMA fills the missing rows with zeros), so
+// one 128 x NB x 64 MMA consumes one 16 KB weight box. The K range of each
+// row tile is split over several CTAs so that about two CTAs per SM stream
+// weights; each CTA stores its fp32 partial tile and the last CTA of a row
+// tile (a ticket counter) sums the partials in split order and runs the
+// epilogue of the prefill's step: 1/rms, bias, per-head RMSNorm and MRoPE
+// with the K/V rows written into the cache (QKV); residual add and the row
+// sum of squares for the next norm (o-projection, down); SiLU(g) * u
+// (gate/up). The weights of a projection do not depend on the previous
+// kernel, so each projection is launched as a programmatic dependent of it
+// and starts streaming its weights before that kernel has finished.
+#include "q3vl_device.cuh"
+#include "q3vl_internal.h"
+
+namespace q3vl {
+
+namespace {
+
+constexpr int kDecThreads = 192;     // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int kDecMaxB = 256;
+constexpr int kBK = 64;              // K elements per stage (one 128-byte row)
+
+__device__ __forceinline__ void dec_epi_sync() {
+  asm volatile("barrier.sync 1, 128;" ::: "memory");
+}
+
+__device__ __forceinline__ float bf16_to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+struct DecGemmParams {
+  int B, NB, R;          // tokens, MMA N (B rounded up to 16), 128-row blocks per tile
+  int n_k, splits, stages;
+  float* part;           // [tiles][splits][B][128 R] fp32 partial tiles
+  uint32_t* tickets;     // [tiles], zero between launches (the last CTA resets)
+  int32_t* err;
+  // epilogue
+  int64_t N;             // output columns (kQkv: q columns nh*128; kSwiGLU: I)
+  __nv_bfloat16* out;    // [B][N]
+  const __nv_bfloat16* resid;  // [B][N] (kResidual)
+  float* rowsq_out;      // [B][N/128] (kResidual) or null
+  const float* rowsq_in; // [B][rowsq_n] (kQkv, kSwiGLU) or null
+  int rowsq_n;
+  float rowsq_width;
+  const float* inv;      // [B] 1/rms when rowsq_in is null
+  float eps;
+  const float* bias;     // [Ntot] or null (kQkv)
+  const float* q_norm;   // [128] (kQkv)
+  const float* k_norm;   // [128] (kQkv)
+  const float2* cs;      // [B][64] (cos, sin) (kQkv)
+  int n_heads, n_kv;
+  __nv_bfloat16* k_cache;  // [n_seq][cap][nkv*128] (kQkv)
+  __nv_bfloat16* v_cache;
+  int64_t cap;
+  int n_seq;
+  const int32_t* seq;    // [B]
+  const int32_t* len;    // [B]
+};
+
+__device__ __forceinline__ float dec_row_scale(const DecGemmParams& p, int j) {
+  if (p.rowsq_in != nullptr) {
+    float ss = 0.f;
+    for (int t = 0; t < p.rowsq_n; ++t) ss += p.rowsq_in[j * p.rowsq_n + t];
+    return 1.0f / sqrtf(ss / p.rowsq_width + p.eps);
+  }
+  return p.inv[j];
+}
+
+__device__ __forceinline__ bool dec_token_valid(const DecGemmParams& p, int j, int& slot,
+                                                int& row) {
+  slot = p.seq[j];
+  row = p.len[j];
+  return slot >= 0 && slot < p.n_seq && row >= 0 && static_cast<int64_t>(row) < p.cap;
+}
+
+// Final epilogue of one token j of row tile `tile`, one warp: lane l holds
+// features l + 32 i (i < 4) of each 128-row block r.
+template <int EPI>
+__device__ __forceinline__ void dec_epilogue_token(const DecGemmParams& p, int tile, int j,
+                                                   int lane, float (&v)[2][4]) {
+  if constexpr (EPI == static_cast<int>(Epi::kQkv)) {
+    const float s = dec_row_scale(p, j);
+    const int64_t c0 = int64_t(tile) * 128;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[0][i] *= s;
+      if (p.bias != nullptr) v[0][i] += p.bias[c0 + lane + 32 * i];
+    }
+    const bool is_q = tile < p.n_heads, is_k = !is_q && tile < p.n_heads + p.n_kv;
+    if (is_q || is_k) {
+      float ss = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) ss += v[0][i] * v[0][i];
+      ss = warp_sum(ss);
+      const float rn = 1.0f / sqrtf(ss * (1.0f / 128.0f) + p.eps);
+      const float* g = is_q ? p.q_norm : p.k_norm;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[0][i] *= rn * g[lane + 32 * i];
+      // split-half rotation: feature f pairs with f + 64 (i with i + 2)
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const float2 q = p.cs[j * 64 + lane + 32 * i];
+        const float a = v[0][i], b = v[0][i + 2];
+        v[0][i] = a * q.x - b * q.y;
+        v[0][i + 2] = a * q.y + b * q.x;
+      }
+    }
+    if (is_q) {
+      __nv_bfloat16* o = p.out + int64_t(j) * p.N + c0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o[lane + 32 * i] = __float2bfloat16_rn(v[0][i]);
+    } else {
+      int slot, row;
+      if (!dec_token_valid(p, j, slot, row)) {
+        if (lane == 0) record_error(p.err, Q3VL_ERANGE, kWhereDecodeRange);
+        return;
+      }
+      const int g = is_k ? tile - p.n_heads : tile - p.n_heads - p.n_kv;
+      const int64_t dkv = int64_t(p.n_kv) * 128;
+      __nv_bfloat16* dst = (is_k ? p.k_cache : p.v_cache) +
+                           (int64_t(slot) * p.cap + row) * dkv + int64_t(g) * 128;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) dst[lane + 32 * i] = __float2bfloat16_rn(v[0][i]);
+    }
+  } else if constexpr (EPI == static_cast<int>(Epi::kResidual)) {
+    const int64_t c0 = int64_t(tile) * 128;
+    const __nv_bfloat16* r = p.resid + int64_t(j) * p.N + c0;
+    __nv_bfloat16* o = p.out + int64_t(j) * p.N + c0;
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat16 ob = __float2bfloat16_rn(bf16_to_f(r[lane + 32 * i]) + v[0][i]);
+      o[lane + 32 * i] = ob;
+      const float f = bf16_to_f(ob);
+      ss += f * f;
+    }
+    if (p.rowsq_out != nullptr) {
+      ss = warp_sum(ss);
+      if (lane == 0) p.rowsq_out[int64_t(j) * (p.N / 128) + tile] = ss;
+    }
+  } else {  // kSwiGLU: block 0 = gate rows, block 1 = the matching up rows
+    const float s = dec_row_scale(p, j);
+    __nv_bfloat16* o = p.out + int64_t(j) * p.N + int64_t(tile) * 128;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      o[lane + 32 * i] = __float2bfloat16_rn(silu_fast(v[0][i] * s) * (v[1][i] * s));
+  }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kDecThreads, 2)
+decode_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                   DecGemmParams p) {
+  constexpr int R = EPI == static_cast<int>(Epi::kSwiGLU) ? 2 : 1;
+  constexpr uint32_t kABytes = 16384u * R;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  const int S = p.stages;
+  const uint32_t b_bytes = static_cast<uint32_t>(p.NB) * 128u;
+  uint8_t* smA = smem;
+  uint8_t* smB = smem + size_t(S) * kABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smB + size_t(S) * b_bytes);
+  uint64_t* empty = full + S;
+  uint64_t* acc_full = empty + S;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = static_cast<int>(blockIdx.x) / p.splits;
+  const int split = static_cast<int>(blockIdx.x) % p.splits;
+  const int k_lo = static_cast<int>(int64_t(split) * p.n_k / p.splits);
+  const int k_hi = static_cast<int>(int64_t(split + 1) * p.n_k / p.splits);
+  const int n = k_hi - k_lo;
+  uint32_t tcols = 32;
+  while (tcols < static_cast<uint32_t>(p.NB * R)) tcols <<= 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) { mbar_init(full + s, 1); mbar_init(empty + s, 1); }
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmX);
+  }
+  if (warp == 1) {
+    // At most a few dozen columns per CTA for small batches; if an earlier
+    // grid still holds this SM's TMEM the allocation waits for it to finish.
+    tmem_alloc(tmem_slot, tcols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  griddep_launch_dependents();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const int32_t row0 = tile * 128 * R;
+      const int pre = n < S ? n : S;
+      // The weights do not depend on the previous kernel: stream the first
+      // stages' boxes before waiting for it.
+      for (int i = 0; i < pre; ++i) {
+        mbar_arrive_expect_tx(full + i, kABytes + b_bytes);
+        tma_load_2d(smA + size_t(i) * kABytes, &tmW, full + i, (k_lo + i) * kBK, row0);
+      }
+      griddep_wait();
+      for (int i = 0; i < pre; ++i)
+        tma_load_2d(smB + size_t(i) * b_bytes, &tmX, full + i, (k_lo + i) * kBK, 0);
+      int issued = pre;
+      for (int i = pre; i < n; ++i) {
+        const int s = i % S;
+        if (!mbar_wait(empty + s, ((i / S) - 1) & 1, p.err, kWhereDecodeProducer, abort_flag))
+          break;
+        mbar_arrive_expect_tx(full + s, kABytes + b_bytes);
+        tma_load_2d(smA + size_t(s) * kABytes, &tmW, full + s, (k_lo + i) * kBK, row0);
+        tma_load_2d(smB + size_t(s) * b_bytes, &tmX, full + s, (k_lo + i) * kBK, 0);
+        issued = i + 1;
+      }
+      // every issued load lands before the CTA may exit
+      for (int i = issued - S > 0 ? issued - S : 0; i < issued; ++i)
+        mbar_wait(full + (i % S), (i / S) & 1, p.err, kWhereDecodeProducer, nullptr);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t d = tmem_base;
+      const uint32_t idesc = idesc_bf16_f32(128, p.NB, false, false);
+      bool ok = true;
+      for (int i = 0; i < n; ++i) {
+        const int s = i % S;
+        if (!mbar_wait(full + s, (i / S) & 1, p.err, kWhereDecodeMma, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(smA + size_t(s) * kABytes);
+        const uint32_t b0 = smem_u32(smB + size_t(s) * b_bytes);
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          const uint64_t bd = sdesc_sw128(b0 + kk * 32, 16, 1024);
+#pragma unroll
+          for (int r = 0; r < R; ++r)
+            umma_bf16_ss(d + r * p.NB, sdesc_sw128(a0 + r * 16384 + kk * 32, 16, 1024), bd, idesc,
+                         (i | kk) != 0 ? 1u : 0u);
+        }
+        umma_commit(empty + s);
+      }
+      if (ok) umma_commit(acc_full);
+      else *abort_flag = 1;
+    }
+    __syncwarp();
+  } else {
+    // epilogue warps: TMEM lanes 32 q .. 32 q + 31 are weight rows (features)
+    griddep_wait();
+    const int q = warp & 3;
+    const int e = warp - 2;  // 0..3
+    bool ok = true;
+    if (lane == 0) ok = mbar_wait(acc_full, 0, p.err, kWhereDecodeEpilogue, abort_flag);
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    if (!ok) *abort_flag = 1;
+    dec_epi_sync();
+    const bool run = *abort_flag == 0;
+    tc_fence_after();
+    const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
+    float* mine = p.part + (size_t(tile) * p.splits + split) * size_t(p.B) * (128 * R);
+    if (run) {
+#pragma unroll 1
+      for (int r = 0; r < R; ++r) {
+#pragma unroll 1
+        for (int c0 = 0; c0 < p.NB; c0 += 16) {
+          uint32_t u[16];
+          tmem_ld16(tbase + r * p.NB + c0, u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int j = c0 + c;
+            if (j < p.B) mine[size_t(j) * (128 * R) + r * 128 + 32 * q + lane] = __uint_as_float(u[c]);
+          }
+        }
+      }
+      __threadfence();
+    }
+    tc_fence_before();
+    dec_epi_sync();
+    if (run && threadIdx.x == 64) {
+      const uint32_t t = atomicAdd(p.tickets + tile, 1u);
+      const bool last = t == static_cast<uint32_t>(p.splits - 1);
+      if (last) p.tickets[tile] = 0;  // every split has arrived: ready for the next launch
+      *last_flag = last ? 1 : 0;
+    }
+    dec_epi_sync();
+    if (run && *last_flag) {
+      __threadfence();
+      const float* base = p.part + size_t(tile) * p.splits * size_t(p.B) * (128 * R);
+#pragma unroll 1
+      for (int j = e; j < p.B; j += 4) {
+        float v[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll 1
+        for (int s = 0; s < p.splits; ++s) {
+          const float* src = base + (size_t(s) * p.B + j) * (128 * R);
+#pragma unroll
+          for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) v[r][i] += __ldcg(src + r * 128 + lane + 32 * i);
+        }
+        dec_epilogue_token<EPI>(p, tile, j, lane, v);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, tcols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Attention of one new row per sequence over its cache (cortiq-engine
+// qwen3te.rs `Qwen3Encoder::attention_gemm`, the last row of the causal
+// softmax: every cached row and the new row itself, row maximum subtracted).
+// Work items are (token b, KV head g, chunk of kAttnCH cache rows); a
+// persistent grid walks them. Each item forms the scores of the G query
+// heads of KV head g, their local maximum m and sum l (base-2 exponent with
+// log2(e)/sqrt(128) folded into q) and the unnormalised o; the last item of
+// a (b, g) to finish (a ticket counter) merges the chunks:
+//   o = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c,  M = max_c m_c.
+// ---------------------------------------------------------------------------
+constexpr int kAttnCH = 128;
+constexpr int kAttnThreads = 128;
+constexpr int kAttnPart = 132;  // floats per (item, head): o[128], m, l, pad
+
+struct DecAttnParams {
+  const __nv_bfloat16* q;        // [B][nh*128]
+  const __nv_bfloat16* k_cache;  // [n_seq][cap][nkv*128]
+  const __nv_bfloat16* v_cache;
+  int64_t cap;
+  int n_seq;
+  const int32_t* seq;
+  const int32_t* len;
+  int B, nkv;
+  float scale_log2;
+  __nv_bfloat16* o;              // [B][nh*128]
+  float* part;                   // [items][G][kAttnPart]
+  uint32_t* tickets;             // [B][nkv], zero between launches
+};
+
+__device__ __forceinline__ void bf16x8_to_f(const uint4& u, float (&f)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = unpack_bf16x2(w[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+
+template <int G>
+__global__ void __launch_bounds__(kAttnThreads)
+decode_attn_kernel(DecAttnParams p) {
+  __shared__ int s_nc[kDecMaxB];
+  __shared__ int s_pref[kDecMaxB + 1];
+  __shared__ float s_p[G][kAttnCH];
+  __shared__ float s_m[G], s_l[G];
+  __shared__ float s_red[8][G][128];
+  __shared__ int s_last;
+
+  griddep_wait();
+  griddep_launch_dependents();
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int nh = G * p.nkv;
+  const int64_t dkv = int64_t(p.nkv) * 128;
+
+  for (int b = t; b < p.B; b += kAttnThreads) {
+    const int slot = p.seq[b], L = p.len[b];
+    const bool ok = slot >= 0 && slot < p.n_seq && L >= 0 && static_cast<int64_t>(L) < p.cap;
+    s_nc[b] = ok ? (L + kAttnCH) / kAttnCH : 0;  // chunks of rows 0..L
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // exclusive prefix of items per token: lane l owns tokens 8l .. 8l+7
+    int loc[8], sum = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int b = 8 * lane + i;
+      loc[i] = sum;
+      sum += b < p.B ? p.nkv * s_nc[b] : 0;
+    }
+    int inc = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    const int excl = inc - sum;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int b = 8 * lane + i;
+      if (b < p.B) s_pref[b] = excl + loc[i];
+    }
+    if (lane == 31) s_pref[p.B] = inc;
+  }
+  __syncthreads();
+  const int total = s_pref[p.B];
+
+  const int hw = lane >> 4, sub = lane & 15;
+  for (int it = blockIdx.x; it < total; it += gridDim.x) {
+    int lo = 0, hi = p.B - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_pref[mid] <= it) lo = mid;
+      else hi = mid - 1;
+    }
+    const int b = lo;
+    const int nc = s_nc[b];
+    const int loc = it - s_pref[b];
+    const int g = loc / nc, c = loc % nc;
+    const int L1 = p.len[b] + 1;
+    const int j0 = c * kAttnCH;
+    const int n = min(kAttnCH, L1 - j0);
+    const int64_t row0 = int64_t(p.seq[b]) * p.cap + j0;
+    const __nv_bfloat16* kb = p.k_cache + row0 * dkv + int64_t(g) * 128;
+    const __nv_bfloat16* vb = p.v_cache + row0 * dkv + int64_t(g) * 128;
+
+    // this lane's 8 dimensions of each query head, scaled
+    float qr[G][8];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const uint4 u = *reinterpret_cast<const uint4*>(p.q + int64_t(b) * nh * 128 +
+                                                      int64_t(g * G + h) * 128 + sub * 8);
+      bf16x8_to_f(u, qr[h]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) qr[h][e] *= p.scale_log2;
+    }
+    // scores: half-warp hw of warp w takes rows 2w + hw + 8r
+#pragma unroll 1
+    for (int r0 = 0; r0 < kAttnCH / 8; r0 += 4) {
+      uint4 kv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int kk = 2 * warp + hw + 8 * (r0 + u);
+        kv[u] = kk < n ? __ldg(reinterpret_cast<const uint4*>(kb + kk * dkv + sub * 8))
+                       : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int kk = 2 * warp + hw + 8 * (r0 + u);
+        float kf[8];
+        bf16x8_to_f(kv[u], kf);
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          float d = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) d = fmaf(qr[h][e], kf[e], d);
+#pragma unroll
+          for (int o = 8; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+          if (sub == 0 && kk < n) s_p[h][kk] = d;
+        }
+      }
+    }
+    __syncthreads();
+    for (int h = warp; h < G; h += 4) {
+      float m = -INFINITY;
+      for (int kk = lane; kk < n; kk += 32) m = fmaxf(m, s_p[h][kk]);
+      m = warp_max(m);
+      float l = 0.f;
+      for (int kk = lane; kk < n; kk += 32) {
+        const float e = ex2_approx(s_p[h][kk] - m);
+        s_p[h][kk] = e;
+        l += e;
+      }
+      l = warp_sum(l);
+      if (lane == 0) { s_m[h] = m; s_l[h] = l; }
+    }
+    __syncthreads();
+    // o: thread t takes dimensions 8 (t % 16) .. +7 of rows t / 16 + 8 r
+    const int dsub = t & 15, ks = t >> 4;
+    float acc[G][8];
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[h][e] = 0.f;
+#pragma unroll 1
+    for (int kk0 = ks; kk0 < n; kk0 += 32) {
+      uint4 vv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int kk = kk0 + 8 * u;
+        vv[u] = kk < n ? __ldg(reinterpret_cast<const uint4*>(vb + kk * dkv + dsub * 8))
+                       : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int kk = kk0 + 8 * u;
+        if (kk < n) {
+          float vf[8];
+          bf16x8_to_f(vv[u], vf);
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float pw = s_p[h][kk];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[h][e] = fmaf(pw, vf[e], acc[h][e]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s_red[ks][h][dsub * 8 + e] = acc[h][e];
+    __syncthreads();
+    __nv_bfloat16* ob = p.o + int64_t(b) * nh * 128 + int64_t(g) * G * 128;
+#pragma unroll 1
+    for (int h = 0; h < G; ++h) {
+      float ov = 0.f;
+#pragma unroll
+      for (int r = 0; r < 8; ++r) ov += s_red[r][h][t];
+      if (nc == 1) {
+        ob[h * 128 + t] = __float2bfloat16_rn(ov / s_l[h]);
+      } else {
+        float* dst = p.part + (size_t(it) * G + h) * kAttnPart;
+        dst[t] = ov;
+        if (t == 0) { dst[128] = s_m[h]; dst[129] = s_l[h]; }
+      }
+    }
+    if (nc > 1) {
+      __threadfence();
+      __syncthreads();
+      if (t == 0) {
+        const uint32_t k = atomicAdd(p.tickets + b * p.nkv + g, 1u);
+        s_last = k == static_cast<uint32_t>(nc - 1);
+        if (s_last) p.tickets[b * p.nkv + g] = 0;
+      }
+      __syncthreads();
+      if (s_last) {
+        __threadfence();
+        const size_t first = size_t(s_pref[b]) + size_t(g) * nc;
+#pragma unroll 1
+        for (int h = 0; h < G; ++h) {
+          float M = -INFINITY;
+          for (int cc = 0; cc < nc; ++cc)
+            M = fmaxf(M, __ldcg(p.part + ((first + cc) * G + h) * kAttnPart + 128));
+          float den = 0.f, num = 0.f;
+          for (int cc = 0; cc < nc; ++cc) {
+            const float* src = p.part + ((first + cc) * G + h) * kAttnPart;
+            const float w = ex2_approx(__ldcg(src + 128) - M);
+            den = fmaf(w, __ldcg(src + 129), den);
+            num = fmaf(w, __ldcg(src + t), num);
+          }
+          ob[h * 128 + t] = __float2bfloat16_rn(num / den);
+        }
+      }
+    }
+    __syncthreads();  // shared buffers are reused by the next item
+  }
+}
+
+// K/V rows of a prefill (the k and v column ranges of the [S, Ntot] QKV
+// buffer) into rows row0 .. row0+S-1 of a cache, 16 bytes per thread.
+__global__ void kv_store_kernel(const uint4* __restrict__ qkv, int64_t S, int64_t ntot8,
+                                int64_t dq8, int64_t dkv8, uint4* __restrict__ k,
+                                uint4* __restrict__ v, int64_t row0) {
+  const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= S * 2 * dkv8) return;
+  const int64_t r = idx / (2 * dkv8), c = idx % (2 * dkv8);
+  const uint4 val = qkv[r * ntot8 + dq8 + c];
+  if (c < dkv8) k[(row0 + r) * dkv8 + c] = val;
+  else v[(row0 + r) * dkv8 + (c - dkv8)] = val;
+}
+
+// Next text token: len[b] + 1, and every position axis + 1.
+__global__ void decode_advance_kernel(int B, int32_t* __restrict__ pos, int32_t* __restrict__ len) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= B) return;
+  len[b] += 1;
+  pos[b] += 1;
+  pos[B + b] += 1;
+  pos[2 * B + b] += 1;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+DecSched dec_gemm_sched(int64_t rows, int64_t K, int B, int R) {
+  DecSched s{};
+  s.R = R;
+  s.NB = (B + 15) / 16 * 16;
+  s.tiles = static_cast<int>(rows / (128 * R));
+  s.n_k = static_cast<int>((K + kBK - 1) / kBK);
+  const size_t stage = size_t(16384) * R + size_t(s.NB) * 128;
+  // up to ~110 KB of stages, so that two CTAs share an SM
+  int st = static_cast<int>(size_t(110 * 1024) / stage);
+  s.stages = st < 2 ? 2 : (st > 8 ? 8 : st);
+  s.smem = 1024 + size_t(s.stages) * stage + size_t(2 * s.stages + 1) * 8 + 16;
+  uint32_t tcols = 32;
+  while (tcols < static_cast<uint32_t>(s.NB * R)) tcols <<= 1;
+  const int resident = (s.smem <= 113 * 1024 && 2 * tcols <= 512) ? 2 : 1;
+  // about `resident` CTAs per SM, one wave; fewer splits when the fp32
+  // partials (written once, read once) would rival the weight bytes
+  int splits = resident * sm_count() / (s.tiles > 0 ? s.tiles : 1);
+  const int64_t by_traffic = K / (8 * int64_t(B));
+  if (splits > by_traffic) splits = static_cast<int>(by_traffic);
+  if (splits > s.n_k) splits = s.n_k;
+  s.splits = splits < 1 ? 1 : splits;
+  return s;
+}
+
+DecLayout dec_layout(const q3vl_config& c, int B, int64_t cap) {
+  DecLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  const int64_t H = c.hidden, I = c.intermediate, Dq = q_dim(c);
+  L.cos_sin = take(size_t(B) * kHalf * 2 * sizeof(float));
+  L.inv = take(size_t(B) * sizeof(float));
+  L.rowsq_h = take(size_t(B) * (H / 128) * sizeof(float));
+  L.rowsq_x = take(size_t(B) * (H / 128) * sizeof(float));
+  L.q = take(size_t(B) * Dq * 2);
+  L.o = take(size_t(B) * Dq * 2);
+  L.h = take(size_t(B) * H * 2);
+  L.act = take(size_t(B) * I * 2);
+  const DecSched sc[4] = {dec_gemm_sched(qkv_dim(c), H, B, 1), dec_gemm_sched(H, Dq, B, 1),
+                          dec_gemm_sched(2 * I, H, B, 2), dec_gemm_sched(H, I, B, 1)};
+  size_t part = 0;
+  int tiles = 0;
+  for (const DecSched& s : sc) {
+    const size_t b = size_t(s.tiles) * s.splits * B * 128 * s.R * sizeof(float);
+    if (b > part) part = b;
+    if (s.tiles > tiles) tiles = s.tiles;
+  }
+  L.part = take(part);
+  const int G = c.n_heads / c.n_kv_heads;
+  L.att_items = int64_t(B) * c.n_kv_heads * ((cap + kAttnCH - 1) / kAttnCH);
+  L.att_part = take(size_t(L.att_items) * G * kAttnPart * sizeof(float));
+  // the two ticket regions come last, so one memset clears both
+  L.tickets = take(size_t(tiles) * sizeof(uint32_t));
+  L.att_tickets = take(size_t(B) * c.n_kv_heads * sizeof(uint32_t));
+  L.total = off;
+  return L;
+}
+
+namespace {
+
+template <typename K, typename... Args>
+cudaError_t launch_pdl(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+template <int EPI>
+cudaError_t launch_dec_epi(const DecGemmArgs& a, int R, cudaStream_t st) {
+  const DecSched s = dec_gemm_sched(a.rows, a.K, a.B, R);
+  static size_t smem_set = 0;  // per instantiation
+  if (s.smem > smem_set) {
+    const cudaError_t e = cudaFuncSetAttribute(
+        decode_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(s.smem));
+    if (e != cudaSuccess) return e;
+    smem_set = s.smem;
+  }
+  CUtensorMap tmW, tmX;
+  if (!make_tmap_bf16(&tmW, a.W, a.rows, a.K, a.K, kBK, 128 * R) ||
+      !make_tmap_bf16(&tmX, a.X, a.B, a.K, a.K, kBK, s.NB))
+    return cudaErrorInvalidValue;
+  DecGemmParams p{};
+  p.B = a.B; p.NB = s.NB; p.R = R;
+  p.n_k = s.n_k; p.splits = s.splits; p.stages = s.stages;
+  p.part = a.part; p.tickets = a.tickets; p.err = device_error_ptr();
+  p.N = a.N; p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.resid = static_cast<const __nv_bfloat16*>(a.resid);
+  p.rowsq_out = a.rowsq_out; p.rowsq_in = a.rowsq_in; p.rowsq_n = a.rowsq_n;
+  p.rowsq_width = a.rowsq_width; p.inv = a.inv; p.eps = a.eps;
+  p.bias = a.bias; p.q_norm = a.q_norm; p.k_norm = a.k_norm;
+  p.cs = reinterpret_cast<const float2*>(a.cos_sin);
+  p.n_heads = a.n_heads; p.n_kv = a.n_kv;
+  p.k_cache = static_cast<__nv_bfloat16*>(a.k_cache);
+  p.v_cache = static_cast<__nv_bfloat16*>(a.v_cache);
+  p.cap = a.cap; p.n_seq = a.n_seq; p.seq = a.seq; p.len = a.len;
+  const cudaError_t e = launch_pdl(decode_gemm_kernel<EPI>, dim3(s.tiles * s.splits),
+                                   dim3(kDecThreads), s.smem, st, tmW, tmX, p);
+  if (e != cudaSuccess) return e;
+  return counted_launch(1);
+}
+
+template <int G>
+cudaError_t launch_attn_g(const DecAttnParams& p, int grid, cudaStream_t st) {
+  const cudaError_t e = launch_pdl(decode_attn_kernel<G>, dim3(grid), dim3(kAttnThreads), 0, st, p);
+  if (e != cudaSuccess) return e;
+  return counted_launch(1);
+}
+
+}  // namespace
+
+cudaError_t launch_decode_gemm(Epi epi, const DecGemmArgs& a, cudaStream_t st) {
+  switch (epi) {
+    case Epi::kQkv: return launch_dec_epi<static_cast<int>(Epi::kQkv)>(a, 1, st);
+    case Epi::kResidual: return launch_dec_epi<static_cast<int>(Epi::kResidual)>(a, 1, st);
+    case Epi::kSwiGLU: return launch_dec_epi<static_cast<int>(Epi::kSwiGLU)>(a, 2, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_decode_attention(const q3vl_config& c, const void* q, const q3vl_kv_cache& kv,
+                                    const int32_t* seq, const int32_t* len, int B, void* o,
+                                    float* part, uint32_t* tickets, int64_t items,
+                                    cudaStream_t st) {
+  DecAttnParams p{};
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k_cache = static_cast<const __nv_bfloat16*>(kv.k);
+  p.v_cache = static_cast<const __nv_bfloat16*>(kv.v);
+  p.cap = kv.cap; p.n_seq = kv.n_seq; p.seq = seq; p.len = len;
+  p.B = B; p.nkv = c.n_kv_heads;
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / 11.313708498984761);  // log2(e)/sqrt(128)
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.part = part; p.tickets = tickets;
+  const int64_t cap_grid = 4 * int64_t(sm_count());
+  const int grid = static_cast<int>(items < cap_grid ? (items > 0 ? items : 1) : cap_grid);
+  switch (c.n_heads / c.n_kv_heads) {
+    case 1: return launch_attn_g<1>(p, grid, st);
+    case 2: return launch_attn_g<2>(p, grid, st);
+    case 4: return launch_attn_g<4>(p, grid, st);
+    case 8: return launch_attn_g<8>(p, grid, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_kv_store(const q3vl_config& c, const void* qkv, int64_t S,
+                            const q3vl_kv_cache& kv, int32_t seq, cudaStream_t st) {
+  const int64_t dkv8 = kv_dim(c) / 8, n = S * 2 * dkv8;
+  kv_store_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
+      static_cast<const uint4*>(qkv), S, qkv_dim(c) / 8, q_dim(c) / 8, dkv8,
+      static_cast<uint4*>(kv.k), static_cast<uint4*>(kv.v), int64_t(seq) * kv.cap);
+  return counted_launch(1);
+}
+
+cudaError_t launch_decode_advance(int B, int32_t* pos, int32_t* len, cudaStream_t st) {
+  decode_advance_kernel<<<(B + 127) / 128, 128, 0, st>>>(B, pos, len);
+  return counted_launch(1);
+}
+
+}  // namespace q3vl

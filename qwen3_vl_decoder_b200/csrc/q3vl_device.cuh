@@ -20,6 +20,8 @@ enum WhereTag : int32_t {
   kWhereGemmProducer = 101, kWhereGemmMma = 102, kWhereGemmEpilogue = 103, kWhereGemmDrain = 104,
   kWhereAttnProducer = 201, kWhereAttnMma = 202, kWhereAttnSoftmax = 203, kWhereAttnDrain = 204,
   kWherePositions = 301, kWhereDeepstackMap = 302, kWhereSelftest = 401,
+  kWhereDecodeProducer = 501, kWhereDecodeMma = 502, kWhereDecodeEpilogue = 503,
+  kWhereDecodeRange = 504, kWhereDecodeAttn = 505,
 };
 
 // Error record: [0] = status code, [1] = location tag. First error wins.
@@ -91,6 +93,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_
       return false;
     }
   }
+}
+
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch (kernels launched with the programmatic
+// stream-serialization attribute)
+// ---------------------------------------------------------------------------
+// Blocks this thread until every grid this one depends on has completed and
+// its memory is visible. A no-op for a grid launched without the attribute.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// Lets the next grid in the stream start its prologue once every CTA of this
+// grid has called this (or exited). The next grid still waits for this one
+// to complete before it reads what this one writes (griddep_wait).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -310,6 +328,17 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
       "r"(r[15])
       : "memory");
+}
+
+// Warp-collective: this warp's 32 TMEM lanes, 16 consecutive fp32 columns.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
 }
 
 __device__ __forceinline__ void tmem_ld_wait() {

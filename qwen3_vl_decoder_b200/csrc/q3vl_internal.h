@@ -126,6 +126,70 @@ cudaError_t launch_gemm_swiglu_f32(const float* A, const float* B, int64_t M, in
 cudaError_t launch_attention_f32(const q3vl_config& c, const float* qkv, int64_t S, float* o,
                                  cudaStream_t st);
 
+// One-token decode (bf16, tcgen05). Schedule of a skinny projection: row
+// tiles of 128 R weight rows, each split over `splits` CTAs along K.
+struct DecSched {
+  int R = 1, NB = 16, tiles = 0, n_k = 0, stages = 2, splits = 1;
+  size_t smem = 0;
+};
+DecSched dec_gemm_sched(int64_t rows, int64_t K, int B, int R);
+
+// Offsets (bytes) of the decode workspace regions.
+struct DecLayout {
+  size_t cos_sin = 0;   // fp32 [B][64][2]
+  size_t inv = 0;       // fp32 [B] input-norm 1/rms of the first layer
+  size_t rowsq_h = 0;   // fp32 [B][H/128] sums of squares of h per 128 columns
+  size_t rowsq_x = 0;   // fp32 [B][H/128] the same of x' (read by the next layer)
+  size_t q = 0;         // bf16 [B][Dq]
+  size_t o = 0;         // bf16 [B][Dq]
+  size_t h = 0;         // bf16 [B][H]
+  size_t act = 0;       // bf16 [B][I]
+  size_t part = 0;      // fp32 partial tiles of the split projections
+  size_t att_part = 0;  // fp32 [att_items][G][132] attention chunk partials
+  size_t tickets = 0;   // uint32 [max tiles], zero between launches
+  size_t att_tickets = 0;  // uint32 [B][nkv], zero between launches
+  int64_t att_items = 0;
+  size_t total = 0;
+};
+DecLayout dec_layout(const q3vl_config& c, int B, int64_t cap);
+
+struct DecGemmArgs {
+  const void* W;        // bf16 [rows, K] weights (row tiles of 128 R)
+  int64_t rows, K;
+  const void* X;        // bf16 [B, K] tokens
+  int B;
+  float* part;
+  uint32_t* tickets;
+  int64_t N;            // output row stride / columns
+  void* out;
+  const void* resid;
+  float* rowsq_out;
+  const float* rowsq_in;
+  int rowsq_n;
+  float rowsq_width;
+  const float* inv;
+  float eps;
+  const float* bias;
+  const float* q_norm;
+  const float* k_norm;
+  const float* cos_sin;
+  int n_heads, n_kv;
+  void* k_cache;
+  void* v_cache;
+  int64_t cap;
+  int n_seq;
+  const int32_t* seq;
+  const int32_t* len;
+};
+cudaError_t launch_decode_gemm(Epi epi, const DecGemmArgs& a, cudaStream_t st);
+cudaError_t launch_decode_attention(const q3vl_config& c, const void* q, const q3vl_kv_cache& kv,
+                                    const int32_t* seq, const int32_t* len, int B, void* o,
+                                    float* part, uint32_t* tickets, int64_t items,
+                                    cudaStream_t st);
+cudaError_t launch_kv_store(const q3vl_config& c, const void* qkv, int64_t S,
+                            const q3vl_kv_cache& kv, int32_t seq, cudaStream_t st);
+cudaError_t launch_decode_advance(int B, int32_t* pos, int32_t* len, cudaStream_t st);
+
 // Device count of SMs (cached per device).
 int sm_count();
 

@@ -128,3 +128,48 @@ def test_positions_argument_checks(lib):
     rc = lib.q3vl_mrope_positions(ctypes.c_void_p(256), 8, None, 1, ctypes.c_void_p(256),
                                   ctypes.c_void_p(256), None)
     assert rc == -1
+
+
+def _kv(cap=64, n_seq=2):
+    from qwen3_vl_decoder_b200 import _abi
+    return _abi.KvCache(256, 512, cap, n_seq)
+
+
+def test_decode_workspace_sizes(lib):
+    c = _cfg()
+    H, Dq, I, nkv, G = 2560, 4096, 9728, 8, 4
+    for B, cap in ((1, 4097), (40, 1000)):
+        ws = lib.q3vl_decode_workspace_bytes(ctypes.byref(c), B, cap)
+        # activations (bf16 q, o, h, act), rope table, norms, attention chunk partials
+        floor = 2 * B * (2 * Dq + H + I) + B * 64 * 8 + B * nkv * -(-cap // 128) * G * 132 * 4
+        assert floor < ws < floor + 64 * 1024 * 1024
+    assert lib.q3vl_decode_workspace_bytes(ctypes.byref(c), 0, 64) == 0
+    assert lib.q3vl_decode_workspace_bytes(ctypes.byref(c), 257, 64) == 0
+    assert lib.q3vl_decode_workspace_bytes(ctypes.byref(c), 1, 0) == 0
+    assert lib.q3vl_decode_workspace_bytes(ctypes.byref(_cfg(dtype="fp32")), 1, 64) == 0
+    assert lib.q3vl_decode_workspace_bytes(ctypes.byref(_cfg(n_heads=48, n_kv_heads=3)), 1, 64) == 0
+
+
+def test_decode_argument_checks(lib):
+    from qwen3_vl_decoder_b200 import _abi
+    c = _cfg()
+    lay = _abi.Layer(*[256] * 7)
+    kv = _kv()
+    P = ctypes.c_void_p(256)
+
+    def dec(B=2, ws_bytes=1 << 40, kv_=kv, cfg=c):
+        return lib.q3vl_layer_decode(ctypes.byref(cfg), ctypes.byref(lay), P, B, P,
+                                     ctypes.byref(kv_), P, P, P, ws_bytes, None)
+    assert dec(B=0) == -1
+    assert dec(B=257) == -1
+    assert dec(ws_bytes=1024) == -5
+    assert dec(kv_=_kv(cap=0)) == -1
+    assert dec(cfg=_cfg(dtype="fp32")) == -8
+    assert lib.q3vl_decode_advance(0, P, P, None) == -1
+    # prefill into a cache: S above the capacity, or a slot outside [0, n_seq)
+    pk = lambda S, seq: lib.q3vl_layer_prefill_kv(ctypes.byref(c), ctypes.byref(lay), P, S, P,
+                                                  None, None, 0, ctypes.byref(kv), seq, P,
+                                                  1 << 40, None)
+    assert pk(65, 0) == -2
+    assert pk(8, 2) == -2
+    assert pk(8, -1) == -2
