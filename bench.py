@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--workload", default=syn.Q4B_LAYER.name, choices=sorted(syn.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="skip the one-token decode measurement of the 36-layer stack")
     return ap.parse_args()
 
 
@@ -316,6 +318,94 @@ def reference_arm(args, w):
     print(json.dumps(line), flush=True)
 
 
+def decode_leg(dev, steps, warmup, batches=(1, 32), w=None):
+    """One-token decode through the 36-layer 4B-shape stack after a 4096-row prompt.
+
+    The prompt is prefilled into slot 0 of every layer's cache (q3vl_stack_prefill_kv)
+    and copied to the other slots. One decode step (a static input copied into x, the
+    36-layer q3vl_stack_decode, q3vl_decode_advance) is captured in a CUDA graph and
+    replayed; the context grows by one row per step. Bytes per step are the packed
+    projection weights of every layer plus each token's cache rows (K and V of all
+    rows up to and including its own), which bound the step by HBM bandwidth.
+    """
+    import qwen3_vl_decoder_b200 as q3
+    w = syn.Q4B_DECODE if w is None else w
+    cfg = q3.config_of(w)
+    layers = []
+    for l in range(w.n_layers):
+        raw = syn.layer_weights(w, l, device=dev)
+        layers.append(q3.pack_layer(cfg, raw))
+        del raw
+    S, Bmax = w.seq, max(batches)
+    cap = S + warmup + steps + 16
+    kvs = q3.kv_caches(cfg, w.n_layers, n_seq=Bmax, cap=cap, device=dev)
+    tt = torch.tensor(syn.token_types(w), dtype=torch.uint8, device=dev)
+    g = syn.grids(w)
+    gd = torch.tensor(g, dtype=torch.int32, device=dev).reshape(-1, 3)
+    pos_p, nxt = q3.mrope_positions(tt, gd)
+    q3.stack_prefill_kv(cfg, layers, syn.hidden_input(w, dev), pos_p, kvs, 0)
+    for kv in kvs:
+        kv.k[1:, :S].copy_(kv.k[0, :S].expand(Bmax - 1, -1, -1))
+        kv.v[1:, :S].copy_(kv.v[0, :S].expand(Bmax - 1, -1, -1))
+    q3.check_device()
+    w_bytes = q3.packed_layer_bytes(cfg)
+    dkv_bytes = 2 * 2 * w.n_kv_heads * w.head_dim          # K and V of one row, bf16
+    out = {"workload": w.name, "prompt_rows": S, "layers": w.n_layers}
+    burst, sustained, hbm, src = peaks()
+    for B in batches:
+        gen = torch.Generator(device=dev).manual_seed(17)
+        x_in = torch.randn(B, w.hidden, generator=gen, device=dev).to(torch.bfloat16)
+        x = torch.empty_like(x_in)
+        seq = torch.arange(B, dtype=torch.int32, device=dev)
+        ws = q3.decode_workspace(cfg, B, cap, dev)
+
+        def reset():
+            return (torch.full((3, B), nxt, dtype=torch.int32, device=dev),
+                    torch.full((B,), S, dtype=torch.int32, device=dev))
+        pos, lens = reset()
+
+        def step():
+            x.copy_(x_in)
+            q3.stack_decode(cfg, layers, x, pos, kvs, seq, lens, None, ws)
+            q3.decode_advance(pos, lens)
+        n0 = q3.launch_count()
+        step()
+        launches = q3.launch_count() - n0
+        torch.cuda.synchronize()
+        p0, l0 = reset()
+        pos.copy_(p0)
+        lens.copy_(l0)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        for _ in range(warmup):
+            graph.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(steps):
+            graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        q3.check_device()
+        assert torch.isfinite(x.float()).all(), "non-finite decode output"
+        t = e0.elapsed_time(e1) / 1e3
+        ctx_mean = S + warmup + (steps - 1) / 2.0          # rows cached before the token
+        step_bytes = w.n_layers * (w_bytes + B * (ctx_mean + 1) * dkv_bytes)
+        gbs = step_bytes * steps / t / 1e9
+        out[f"B{B}"] = {"value": B * steps / t, "unit": "tokens/s", "batch": B,
+                        "ms_per_step": 1e3 * t / steps,
+                        "us_per_layer": 1e6 * t / steps / w.n_layers, "steps": steps,
+                        "kernel_launches_per_step": launches,
+                        "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                                     "frac": gbs / hbm, "bytes_per_step": step_bytes,
+                                     "peak_source": f"{src} copy bandwidth"}}
+        del graph
+    del kvs, layers
+    torch.cuda.empty_cache()
+    return out
+
+
 def main():
     args = parse()
     w = syn.WORKLOADS[args.workload]
@@ -390,6 +480,10 @@ def main():
         del st2
         torch.cuda.empty_cache()
 
+    decode = None
+    if world == 1 and not args.no_decode:
+        decode = decode_leg(dev, min(args.steps, 400), max(3, min(args.warmup, 20)))
+
     burst, sustained, hbm, src = peaks()
     gemm_f, attn_f = layer_flops(w)
     H, I = w.hidden, w.intermediate
@@ -442,6 +536,7 @@ def main():
         "e2e": {"value": world * S * args.steps / t_e2e, "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": st["out_host"].numel() * 2},
         "also": also,
+        "decode": decode,
         "gpu_launches": launches,
         "clocks": clk.summary(),
         "next_position": nxt,

@@ -77,6 +77,11 @@ Q32B_ENC_1064 = Q32B_ENC.with_seq(1064)
 WORKLOADS = {w.name: w for w in (TINY_FP32, Q2B_LAYER, Q2B_STACK, Q4B_LAYER, Q32B_ENC,
                                   Q32B_ENC_1064)}
 
+# Decode after a prompt: the 4B shape with its 36 layers, the prompt being the
+# 4B layer workload's (512 text, a 32x24 image, 2816 text = 4096 rows).
+Q4B_DECODE = Workload("qwen3vl-4b-stack36-decode-ctx4096", 2560, 32, 8, 9728, 4096, 36, "bf16",
+                      3, qkv_bias=True, images=((512, 32, 24),))
+
 
 def token_types(w: Workload) -> List[int]:
     """Per-token type: 0 = text, 1 = image placeholder (merged grid token)."""

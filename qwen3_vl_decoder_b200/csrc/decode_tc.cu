@@ -298,28 +298,75 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     }
     tc_fence_before();
     dec_epi_sync();
-    if (run && threadIdx.x == 64) {
-      const uint32_t t = atomicAdd(p.tickets + tile, 1u);
-      const bool last = t == static_cast<uint32_t>(p.splits - 1);
-      if (last) p.tickets[tile] = 0;  // every split has arrived: ready for the next launch
+    if (threadIdx.x == 64) {
+      // one thread decides for the four warps (the barriers below need all four)
+      bool last = false;
+      if (run) {
+        const uint32_t t = atomicAdd(p.tickets + tile, 1u);
+        last = t == static_cast<uint32_t>(p.splits - 1);
+        if (last) p.tickets[tile] = 0;  // every split has arrived: ready for the next launch
+      }
       *last_flag = last ? 1 : 0;
     }
     dec_epi_sync();
-    if (run && *last_flag) {
+    if (*last_flag) {
       __threadfence();
-      const float* base = p.part + size_t(tile) * p.splits * size_t(p.B) * (128 * R);
+      // Sum the splits in split order into shared memory (the drained stage
+      // ring), all 128 threads with up to 16 independent 16-byte loads in
+      // flight each, then run the epilogue one token per warp from there.
+      const float4* base4 = reinterpret_cast<const float4*>(
+          p.part + size_t(tile) * p.splits * size_t(p.B) * (128 * R));
+      float4* red = reinterpret_cast<float4*>(smem);
+      const size_t ring = size_t(S) * (kABytes + b_bytes);
+      const int chunk = static_cast<int>(ring / (512u * R)) < p.B
+                            ? static_cast<int>(ring / (512u * R)) : p.B;
+      const size_t stride4 = size_t(p.B) * (32 * R);  // float4 per split
+      const int et = threadIdx.x - 64;
 #pragma unroll 1
-      for (int j = e; j < p.B; j += 4) {
-        float v[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      for (int j0 = 0; j0 < p.B; j0 += chunk) {
+        const int nj = p.B - j0 < chunk ? p.B - j0 : chunk;
+        const int n4 = nj * 32 * R;
+        const float4* src = base4 + size_t(j0) * (32 * R);
 #pragma unroll 1
-        for (int s = 0; s < p.splits; ++s) {
-          const float* src = base + (size_t(s) * p.B + j) * (128 * R);
+        for (int q0 = et; q0 < n4; q0 += 4 * 128) {
+          float4 acc[4];
 #pragma unroll
-          for (int r = 0; r < R; ++r)
+          for (int u = 0; u < 4; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+          for (int s0 = 0; s0 < p.splits; s0 += 4) {
+            float4 v[4][4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) v[r][i] += __ldcg(src + r * 128 + lane + 32 * i);
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                v[u][k] = (s0 + k < p.splits && q0 + 128 * u < n4)
+                              ? __ldcg(src + size_t(s0 + k) * stride4 + q0 + 128 * u)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                acc[u].x += v[u][k].x; acc[u].y += v[u][k].y;
+                acc[u].z += v[u][k].z; acc[u].w += v[u][k].w;
+              }
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (q0 + 128 * u < n4) red[q0 + 128 * u] = acc[u];
         }
-        dec_epilogue_token<EPI>(p, tile, j, lane, v);
+        dec_epi_sync();
+        const float* redf = reinterpret_cast<const float*>(red);
+#pragma unroll 1
+        for (int j = e; j < nj; j += 4) {
+          float v[2][4];
+#pragma unroll
+          for (int r = 0; r < 2; ++r)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              v[r][i] = r < R ? redf[size_t(j) * (128 * R) + r * 128 + lane + 32 * i] : 0.f;
+          dec_epilogue_token<EPI>(p, tile, j0 + j, lane, v);
+        }
+        dec_epi_sync();
       }
     }
   }
@@ -335,16 +382,18 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
 // Attention of one new row per sequence over its cache (cortiq-engine
 // qwen3te.rs `Qwen3Encoder::attention_gemm`, the last row of the causal
 // softmax: every cached row and the new row itself, row maximum subtracted).
-// Work items are (token b, KV head g, chunk of kAttnCH cache rows); a
-// persistent grid walks them. Each item forms the scores of the G query
-// heads of KV head g, their local maximum m and sum l (base-2 exponent with
-// log2(e)/sqrt(128) folded into q) and the unnormalised o; the last item of
-// a (b, g) to finish (a ticket counter) merges the chunks:
+// Work items are (token b, KV head g, chunk c of kAttnCH cache rows); a
+// persistent grid walks them. An item copies its K and V rows into shared
+// memory (cp.async, all in flight at once), forms the scores of the G query
+// heads of KV head g, their maximum m and sum l (base-2 exponent with
+// log2(e)/sqrt(128) folded into q) and the unnormalised o. With one chunk
+// the item writes o / l; otherwise the last item of a (b, g) to finish (a
+// ticket counter) merges the chunks:
 //   o = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c,  M = max_c m_c.
 // ---------------------------------------------------------------------------
 constexpr int kAttnCH = 128;
 constexpr int kAttnThreads = 128;
-constexpr int kAttnPart = 132;  // floats per (item, head): o[128], m, l, pad
+constexpr int kAttnRows = 130;  // per (b, g, h): o[128], m, l, each over the chunk slots
 
 struct DecAttnParams {
   const __nv_bfloat16* q;        // [B][nh*128]
@@ -355,9 +404,10 @@ struct DecAttnParams {
   const int32_t* seq;
   const int32_t* len;
   int B, nkv;
+  int nc_pad;                    // chunk slots per (b, g): ceil(cap / kAttnCH), rounded up to 4
   float scale_log2;
   __nv_bfloat16* o;              // [B][nh*128]
-  float* part;                   // [items][G][kAttnPart]
+  float* part;                   // [B][nkv][G][kAttnRows][nc_pad]
   uint32_t* tickets;             // [B][nkv], zero between launches
 };
 
@@ -372,14 +422,26 @@ __device__ __forceinline__ void bf16x8_to_f(const uint4& u, float (&f)[8]) {
 }
 
 template <int G>
+__host__ __device__ constexpr size_t attn_smem_bytes(int nc_pad) {
+  return size_t(2) * kAttnCH * 128 * 2 + size_t(G) * kAttnCH * 4 + size_t(2) * G * nc_pad * 4 +
+         size_t(3) * G * 4 + (2 * kDecMaxB + 2) * 4;
+}
+
+template <int G>
 __global__ void __launch_bounds__(kAttnThreads)
 decode_attn_kernel(DecAttnParams p) {
-  __shared__ int s_nc[kDecMaxB];
-  __shared__ int s_pref[kDecMaxB + 1];
-  __shared__ float s_p[G][kAttnCH];
-  __shared__ float s_m[G], s_l[G];
-  __shared__ float s_red[8][G][128];
-  __shared__ int s_last;
+  extern __shared__ __align__(16) uint8_t sm[];
+  __nv_bfloat16* k_s = reinterpret_cast<__nv_bfloat16*>(sm);
+  __nv_bfloat16* v_s = k_s + kAttnCH * 128;
+  float* s_p = reinterpret_cast<float*>(v_s + kAttnCH * 128);   // [G][CH]
+  float* s_w = s_p + G * kAttnCH;                                // [G][nc_pad] maxima, weights
+  float* s_cl = s_w + G * p.nc_pad;                              // [G][nc_pad] chunk sums
+  float* s_m = s_cl + G * p.nc_pad;                              // [G]
+  float* s_l = s_m + G;
+  float* s_den = s_l + G;
+  int* s_nc = reinterpret_cast<int*>(s_den + G);                 // [kDecMaxB]
+  int* s_pref = s_nc + kDecMaxB;                                 // [kDecMaxB + 1]
+  int* s_last = s_pref + kDecMaxB + 1;
 
   griddep_wait();
   griddep_launch_dependents();
@@ -431,13 +493,19 @@ decode_attn_kernel(DecAttnParams p) {
     const int nc = s_nc[b];
     const int loc = it - s_pref[b];
     const int g = loc / nc, c = loc % nc;
-    const int L1 = p.len[b] + 1;
     const int j0 = c * kAttnCH;
-    const int n = min(kAttnCH, L1 - j0);
+    const int n = min(kAttnCH, p.len[b] + 1 - j0);
     const int64_t row0 = int64_t(p.seq[b]) * p.cap + j0;
     const __nv_bfloat16* kb = p.k_cache + row0 * dkv + int64_t(g) * 128;
     const __nv_bfloat16* vb = p.v_cache + row0 * dkv + int64_t(g) * 128;
 
+    // this item's K and V rows -> shared memory, all copies in flight at once
+    for (int idx = t; idx < n * 16; idx += kAttnThreads) {
+      const int r = idx >> 4, piece = idx & 15;
+      cp_async16(k_s + r * 128 + piece * 8, kb + r * dkv + piece * 8);
+      cp_async16(v_s + r * 128 + piece * 8, vb + r * dkv + piece * 8);
+    }
+    cp_async_commit();
     // this lane's 8 dimensions of each query head, scaled
     float qr[G][8];
 #pragma unroll
@@ -448,123 +516,135 @@ decode_attn_kernel(DecAttnParams p) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) qr[h][e] *= p.scale_log2;
     }
-    // scores: half-warp hw of warp w takes rows 2w + hw + 8r
-#pragma unroll 1
-    for (int r0 = 0; r0 < kAttnCH / 8; r0 += 4) {
-      uint4 kv[4];
+    cp_async_wait_all();
+    __syncthreads();
+    // scores: half-warp hw of warp w takes rows 2w + hw + 8r. The trip count
+    // is the same for every lane of the warp (the shuffles need all 32).
+#pragma unroll 2
+    for (int k0 = 2 * warp; k0 < n; k0 += 8) {
+      const int kk = k0 + hw;
+      float kf[8];
+      if (kk < n) {
+        bf16x8_to_f(*reinterpret_cast<const uint4*>(k_s + kk * 128 + sub * 8), kf);
+      } else {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int kk = 2 * warp + hw + 8 * (r0 + u);
-        kv[u] = kk < n ? __ldg(reinterpret_cast<const uint4*>(kb + kk * dkv + sub * 8))
-                       : make_uint4(0, 0, 0, 0);
+        for (int e = 0; e < 8; ++e) kf[e] = 0.f;
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int kk = 2 * warp + hw + 8 * (r0 + u);
-        float kf[8];
-        bf16x8_to_f(kv[u], kf);
+      for (int h = 0; h < G; ++h) {
+        float d = 0.f;
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          float d = 0.f;
+        for (int e = 0; e < 8; ++e) d = fmaf(qr[h][e], kf[e], d);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) d = fmaf(qr[h][e], kf[e], d);
-#pragma unroll
-          for (int o = 8; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-          if (sub == 0 && kk < n) s_p[h][kk] = d;
-        }
+        for (int o = 8; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+        if (sub == 0 && kk < n) s_p[h * kAttnCH + kk] = d;
       }
     }
     __syncthreads();
     for (int h = warp; h < G; h += 4) {
       float m = -INFINITY;
-      for (int kk = lane; kk < n; kk += 32) m = fmaxf(m, s_p[h][kk]);
+      for (int kk = lane; kk < n; kk += 32) m = fmaxf(m, s_p[h * kAttnCH + kk]);
       m = warp_max(m);
       float l = 0.f;
       for (int kk = lane; kk < n; kk += 32) {
-        const float e = ex2_approx(s_p[h][kk] - m);
-        s_p[h][kk] = e;
+        const float e = ex2_approx(s_p[h * kAttnCH + kk] - m);
+        s_p[h * kAttnCH + kk] = e;
         l += e;
       }
       l = warp_sum(l);
       if (lane == 0) { s_m[h] = m; s_l[h] = l; }
     }
     __syncthreads();
-    // o: thread t takes dimensions 8 (t % 16) .. +7 of rows t / 16 + 8 r
-    const int dsub = t & 15, ks = t >> 4;
-    float acc[G][8];
+    // o[h][t] = sum_kk p[h][kk] v[kk][t]
+    float acc[G];
 #pragma unroll
-    for (int h = 0; h < G; ++h)
+    for (int h = 0; h < G; ++h) acc[h] = 0.f;
+    const int n4 = n & ~3;
+#pragma unroll 2
+    for (int kk = 0; kk < n4; kk += 4) {
+      float v[4];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[h][e] = 0.f;
-#pragma unroll 1
-    for (int kk0 = ks; kk0 < n; kk0 += 32) {
-      uint4 vv[4];
+      for (int u = 0; u < 4; ++u) v[u] = __bfloat162float(v_s[(kk + u) * 128 + t]);
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int kk = kk0 + 8 * u;
-        vv[u] = kk < n ? __ldg(reinterpret_cast<const uint4*>(vb + kk * dkv + dsub * 8))
-                       : make_uint4(0, 0, 0, 0);
+      for (int h = 0; h < G; ++h) {
+        const float4 pw = *reinterpret_cast<const float4*>(s_p + h * kAttnCH + kk);
+        acc[h] = fmaf(pw.x, v[0], acc[h]);
+        acc[h] = fmaf(pw.y, v[1], acc[h]);
+        acc[h] = fmaf(pw.z, v[2], acc[h]);
+        acc[h] = fmaf(pw.w, v[3], acc[h]);
       }
+    }
+    for (int kk = n4; kk < n; ++kk) {
+      const float v = __bfloat162float(v_s[kk * 128 + t]);
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int kk = kk0 + 8 * u;
-        if (kk < n) {
-          float vf[8];
-          bf16x8_to_f(vv[u], vf);
+      for (int h = 0; h < G; ++h) acc[h] = fmaf(s_p[h * kAttnCH + kk], v, acc[h]);
+    }
+    __nv_bfloat16* ob = p.o + int64_t(b) * nh * 128 + int64_t(g) * G * 128;
+    float* pb = p.part + (size_t(b) * p.nkv + g) * G * kAttnRows * size_t(p.nc_pad);
+    if (nc == 1) {
 #pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float pw = s_p[h][kk];
+      for (int h = 0; h < G; ++h) ob[h * 128 + t] = __float2bfloat16_rn(acc[h] / s_l[h]);
+    } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[h][e] = fmaf(pw, vf[e], acc[h][e]);
-          }
+      for (int h = 0; h < G; ++h) {
+        float* ph = pb + size_t(h) * kAttnRows * p.nc_pad;
+        ph[size_t(t) * p.nc_pad + c] = acc[h];
+        if (t == 0) {
+          ph[size_t(128) * p.nc_pad + c] = s_m[h];
+          ph[size_t(129) * p.nc_pad + c] = s_l[h];
         }
       }
-    }
-#pragma unroll
-    for (int h = 0; h < G; ++h)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) s_red[ks][h][dsub * 8 + e] = acc[h][e];
-    __syncthreads();
-    __nv_bfloat16* ob = p.o + int64_t(b) * nh * 128 + int64_t(g) * G * 128;
-#pragma unroll 1
-    for (int h = 0; h < G; ++h) {
-      float ov = 0.f;
-#pragma unroll
-      for (int r = 0; r < 8; ++r) ov += s_red[r][h][t];
-      if (nc == 1) {
-        ob[h * 128 + t] = __float2bfloat16_rn(ov / s_l[h]);
-      } else {
-        float* dst = p.part + (size_t(it) * G + h) * kAttnPart;
-        dst[t] = ov;
-        if (t == 0) { dst[128] = s_m[h]; dst[129] = s_l[h]; }
-      }
-    }
-    if (nc > 1) {
       __threadfence();
       __syncthreads();
       if (t == 0) {
         const uint32_t k = atomicAdd(p.tickets + b * p.nkv + g, 1u);
-        s_last = k == static_cast<uint32_t>(nc - 1);
-        if (s_last) p.tickets[b * p.nkv + g] = 0;
+        *s_last = k == static_cast<uint32_t>(nc - 1);
+        if (*s_last) p.tickets[b * p.nkv + g] = 0;
       }
       __syncthreads();
-      if (s_last) {
+      if (*s_last) {
         __threadfence();
-        const size_t first = size_t(s_pref[b]) + size_t(g) * nc;
-#pragma unroll 1
-        for (int h = 0; h < G; ++h) {
-          float M = -INFINITY;
-          for (int cc = 0; cc < nc; ++cc)
-            M = fmaxf(M, __ldcg(p.part + ((first + cc) * G + h) * kAttnPart + 128));
-          float den = 0.f, num = 0.f;
-          for (int cc = 0; cc < nc; ++cc) {
-            const float* src = p.part + ((first + cc) * G + h) * kAttnPart;
-            const float w = ex2_approx(__ldcg(src + 128) - M);
-            den = fmaf(w, __ldcg(src + 129), den);
-            num = fmaf(w, __ldcg(src + t), num);
-          }
-          ob[h * 128 + t] = __float2bfloat16_rn(num / den);
+        // chunk maxima and weights in shared memory, then every thread merges
+        // one dimension of every head with independent 16-byte loads
+        for (int idx = t; idx < G * nc; idx += kAttnThreads) {
+          const int h = idx / nc, cc = idx % nc;
+          s_w[h * p.nc_pad + cc] = __ldcg(pb + (size_t(h) * kAttnRows + 128) * p.nc_pad + cc);
+          s_cl[h * p.nc_pad + cc] = __ldcg(pb + (size_t(h) * kAttnRows + 129) * p.nc_pad + cc);
         }
+        __syncthreads();
+        if (t < G) {
+          float M = -INFINITY;
+          for (int cc = 0; cc < nc; ++cc) M = fmaxf(M, s_w[t * p.nc_pad + cc]);
+          float den = 0.f;
+          for (int cc = 0; cc < nc; ++cc) {
+            const float w = ex2_approx(s_w[t * p.nc_pad + cc] - M);
+            s_w[t * p.nc_pad + cc] = w;
+            den = fmaf(w, s_cl[t * p.nc_pad + cc], den);
+          }
+          s_den[t] = den;
+        }
+        __syncthreads();
+        float num[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) num[h] = 0.f;
+#pragma unroll 4
+        for (int c4 = 0; c4 < nc; c4 += 4) {
+          float4 v[G];
+#pragma unroll
+          for (int h = 0; h < G; ++h)
+            v[h] = __ldcg(reinterpret_cast<const float4*>(
+                pb + (size_t(h) * kAttnRows + t) * p.nc_pad + c4));
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float* wv = s_w + h * p.nc_pad + c4;
+            const float vv[4] = {v[h].x, v[h].y, v[h].z, v[h].w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              if (c4 + u < nc) num[h] = fmaf(wv[u], vv[u], num[h]);
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < G; ++h) ob[h * 128 + t] = __float2bfloat16_rn(num[h] / s_den[h]);
       }
     }
     __syncthreads();  // shared buffers are reused by the next item
@@ -651,8 +731,9 @@ DecLayout dec_layout(const q3vl_config& c, int B, int64_t cap) {
   }
   L.part = take(part);
   const int G = c.n_heads / c.n_kv_heads;
+  const int64_t nc_pad = ((cap + kAttnCH - 1) / kAttnCH + 3) / 4 * 4;
   L.att_items = int64_t(B) * c.n_kv_heads * ((cap + kAttnCH - 1) / kAttnCH);
-  L.att_part = take(size_t(L.att_items) * G * kAttnPart * sizeof(float));
+  L.att_part = take(size_t(B) * c.n_kv_heads * G * kAttnRows * nc_pad * sizeof(float));
   // the two ticket regions come last, so one memset clears both
   L.tickets = take(size_t(tiles) * sizeof(uint32_t));
   L.att_tickets = take(size_t(B) * c.n_kv_heads * sizeof(uint32_t));
@@ -714,7 +795,16 @@ cudaError_t launch_dec_epi(const DecGemmArgs& a, int R, cudaStream_t st) {
 
 template <int G>
 cudaError_t launch_attn_g(const DecAttnParams& p, int grid, cudaStream_t st) {
-  const cudaError_t e = launch_pdl(decode_attn_kernel<G>, dim3(grid), dim3(kAttnThreads), 0, st, p);
+  const size_t smem = attn_smem_bytes<G>(p.nc_pad);
+  static size_t smem_set = 0;  // per instantiation
+  if (smem > smem_set) {
+    const cudaError_t e = cudaFuncSetAttribute(
+        decode_attn_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    smem_set = smem;
+  }
+  const cudaError_t e =
+      launch_pdl(decode_attn_kernel<G>, dim3(grid), dim3(kAttnThreads), smem, st, p);
   if (e != cudaSuccess) return e;
   return counted_launch(1);
 }
@@ -740,6 +830,7 @@ cudaError_t launch_decode_attention(const q3vl_config& c, const void* q, const q
   p.v_cache = static_cast<const __nv_bfloat16*>(kv.v);
   p.cap = kv.cap; p.n_seq = kv.n_seq; p.seq = seq; p.len = len;
   p.B = B; p.nkv = c.n_kv_heads;
+  p.nc_pad = static_cast<int>(((kv.cap + kAttnCH - 1) / kAttnCH + 3) / 4 * 4);
   p.scale_log2 = static_cast<float>(1.4426950408889634 / 11.313708498984761);  // log2(e)/sqrt(128)
   p.o = static_cast<__nv_bfloat16*>(o);
   p.part = part; p.tickets = tickets;
