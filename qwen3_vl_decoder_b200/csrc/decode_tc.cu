@@ -392,7 +392,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
 //   o = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c,  M = max_c m_c.
 // ---------------------------------------------------------------------------
 constexpr int kAttnCH = 128;
-constexpr int kAttnThreads = 128;
+constexpr int kAttnThreads = 256;
 constexpr int kAttnRows = 130;  // per (b, g, h): o[128], m, l, each over the chunk slots
 
 struct DecAttnParams {
@@ -423,18 +423,20 @@ __device__ __forceinline__ void bf16x8_to_f(const uint4& u, float (&f)[8]) {
 
 template <int G>
 __host__ __device__ constexpr size_t attn_smem_bytes(int nc_pad) {
-  return size_t(2) * kAttnCH * 128 * 2 + size_t(G) * kAttnCH * 4 + size_t(2) * G * nc_pad * 4 +
+  return size_t(2) * kAttnCH * 128 * 2 + size_t(G) * kAttnCH * 4 + size_t(G) * 128 * 4 +
+         size_t(2) * G * nc_pad * 4 +
          size_t(3) * G * 4 + (2 * kDecMaxB + 2) * 4;
 }
 
 template <int G>
-__global__ void __launch_bounds__(kAttnThreads)
+__global__ void __launch_bounds__(kAttnThreads, 2)
 decode_attn_kernel(DecAttnParams p) {
   extern __shared__ __align__(16) uint8_t sm[];
   __nv_bfloat16* k_s = reinterpret_cast<__nv_bfloat16*>(sm);
   __nv_bfloat16* v_s = k_s + kAttnCH * 128;
   float* s_p = reinterpret_cast<float*>(v_s + kAttnCH * 128);   // [G][CH]
-  float* s_w = s_p + G * kAttnCH;                                // [G][nc_pad] maxima, weights
+  float* s_red = s_p + G * kAttnCH;                              // [G][128]
+  float* s_w = s_red + G * 128;                                  // [G][nc_pad] maxima, weights
   float* s_cl = s_w + G * p.nc_pad;                              // [G][nc_pad] chunk sums
   float* s_m = s_cl + G * p.nc_pad;                              // [G]
   float* s_l = s_m + G;
@@ -481,7 +483,6 @@ decode_attn_kernel(DecAttnParams p) {
   __syncthreads();
   const int total = s_pref[p.B];
 
-  const int hw = lane >> 4, sub = lane & 15;
   for (int it = blockIdx.x; it < total; it += gridDim.x) {
     int lo = 0, hi = p.B - 1;
     while (lo < hi) {
@@ -506,42 +507,52 @@ decode_attn_kernel(DecAttnParams p) {
       cp_async16(v_s + r * 128 + piece * 8, vb + r * dkv + piece * 8);
     }
     cp_async_commit();
-    // this lane's 8 dimensions of each query head, scaled
-    float qr[G][8];
+    // Scores: a group of LPK = 2G lanes per cache row, each lane holding D =
+    // 64/G dimensions of every query head (64 values of q per lane).
+    constexpr int LPK = 2 * G, D = 128 / LPK, KPW = 32 / LPK;
+    const int kl = lane % LPK, kr = lane / LPK;
+    float qr[G][D];
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const uint4 u = *reinterpret_cast<const uint4*>(p.q + int64_t(b) * nh * 128 +
-                                                      int64_t(g * G + h) * 128 + sub * 8);
-      bf16x8_to_f(u, qr[h]);
+    for (int h = 0; h < G; ++h)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) qr[h][e] *= p.scale_log2;
-    }
+      for (int e = 0; e < D / 8; ++e) {
+        float f[8];
+        bf16x8_to_f(*reinterpret_cast<const uint4*>(p.q + int64_t(b) * nh * 128 +
+                                                   int64_t(g * G + h) * 128 + kl * D + 8 * e),
+                    f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) qr[h][8 * e + i] = f[i] * p.scale_log2;
+      }
     cp_async_wait_all();
     __syncthreads();
-    // scores: half-warp hw of warp w takes rows 2w + hw + 8r. The trip count
-    // is the same for every lane of the warp (the shuffles need all 32).
-#pragma unroll 2
-    for (int k0 = 2 * warp; k0 < n; k0 += 8) {
-      const int kk = k0 + hw;
-      float kf[8];
+    // the trip count depends on the warp only (the shuffles need all 32 lanes)
+#pragma unroll 1
+    for (int k0 = KPW * warp; k0 < n; k0 += KPW * (kAttnThreads / 32)) {
+      const int kk = k0 + kr;
+      float d[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) d[h] = 0.f;
       if (kk < n) {
-        bf16x8_to_f(*reinterpret_cast<const uint4*>(k_s + kk * 128 + sub * 8), kf);
-      } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) kf[e] = 0.f;
+        for (int e = 0; e < D / 8; ++e) {
+          float kf[8];
+          bf16x8_to_f(*reinterpret_cast<const uint4*>(k_s + kk * 128 + kl * D + 8 * e), kf);
+#pragma unroll
+          for (int h = 0; h < G; ++h)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) d[h] = fmaf(qr[h][8 * e + i], kf[i], d[h]);
+        }
       }
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float d = 0.f;
+      for (int h = 0; h < G; ++h)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) d = fmaf(qr[h][e], kf[e], d);
+        for (int o = LPK / 2; o > 0; o >>= 1) d[h] += __shfl_xor_sync(0xffffffffu, d[h], o);
+      if (kl == 0 && kk < n)
 #pragma unroll
-        for (int o = 8; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-        if (sub == 0 && kk < n) s_p[h * kAttnCH + kk] = d;
-      }
+        for (int h = 0; h < G; ++h) s_p[h * kAttnCH + kk] = d[h];
     }
     __syncthreads();
-    for (int h = warp; h < G; h += 4) {
+    for (int h = warp; h < G; h += kAttnThreads / 32) {
       float m = -INFINITY;
       for (int kk = lane; kk < n; kk += 32) m = fmaxf(m, s_p[h * kAttnCH + kk]);
       m = warp_max(m);
@@ -555,45 +566,61 @@ decode_attn_kernel(DecAttnParams p) {
       if (lane == 0) { s_m[h] = m; s_l[h] = l; }
     }
     __syncthreads();
-    // o[h][t] = sum_kk p[h][kk] v[kk][t]
+    // o[h][d] = sum_kk p[h][kk] v[kk][d]: thread t takes dimension t % 128 over
+    // rows [64 (t / 128), 64 (t / 128) + 64) of the chunk; the halves meet in
+    // shared memory
+    const int dd = t & 127, half = t >> 7;
     float acc[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) acc[h] = 0.f;
-    const int n4 = n & ~3;
+    {
+      const int kbeg = half * (kAttnCH / 2);
+      const int kend = min(n, kbeg + kAttnCH / 2);
+      int kk = kbeg;
 #pragma unroll 2
-    for (int kk = 0; kk < n4; kk += 4) {
-      float v[4];
+      for (; kk + 4 <= kend; kk += 4) {
+        float v[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = __bfloat162float(v_s[(kk + u) * 128 + t]);
+        for (int u = 0; u < 4; ++u) v[u] = __bfloat162float(v_s[(kk + u) * 128 + dd]);
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float4 pw = *reinterpret_cast<const float4*>(s_p + h * kAttnCH + kk);
-        acc[h] = fmaf(pw.x, v[0], acc[h]);
-        acc[h] = fmaf(pw.y, v[1], acc[h]);
-        acc[h] = fmaf(pw.z, v[2], acc[h]);
-        acc[h] = fmaf(pw.w, v[3], acc[h]);
+        for (int h = 0; h < G; ++h) {
+          const float4 pw = *reinterpret_cast<const float4*>(s_p + h * kAttnCH + kk);
+          acc[h] = fmaf(pw.x, v[0], acc[h]);
+          acc[h] = fmaf(pw.y, v[1], acc[h]);
+          acc[h] = fmaf(pw.z, v[2], acc[h]);
+          acc[h] = fmaf(pw.w, v[3], acc[h]);
+        }
+      }
+      for (; kk < kend; ++kk) {
+        const float v = __bfloat162float(v_s[kk * 128 + dd]);
+#pragma unroll
+        for (int h = 0; h < G; ++h) acc[h] = fmaf(s_p[h * kAttnCH + kk], v, acc[h]);
       }
     }
-    for (int kk = n4; kk < n; ++kk) {
-      const float v = __bfloat162float(v_s[kk * 128 + t]);
+    if (half == 1)
 #pragma unroll
-      for (int h = 0; h < G; ++h) acc[h] = fmaf(s_p[h * kAttnCH + kk], v, acc[h]);
-    }
+      for (int h = 0; h < G; ++h) s_red[h * 128 + dd] = acc[h];
+    __syncthreads();
+    if (half == 0)
+#pragma unroll
+      for (int h = 0; h < G; ++h) acc[h] += s_red[h * 128 + dd];
     __nv_bfloat16* ob = p.o + int64_t(b) * nh * 128 + int64_t(g) * G * 128;
     float* pb = p.part + (size_t(b) * p.nkv + g) * G * kAttnRows * size_t(p.nc_pad);
     if (nc == 1) {
+      if (half == 0)
 #pragma unroll
-      for (int h = 0; h < G; ++h) ob[h * 128 + t] = __float2bfloat16_rn(acc[h] / s_l[h]);
+        for (int h = 0; h < G; ++h) ob[h * 128 + dd] = __float2bfloat16_rn(acc[h] / s_l[h]);
     } else {
+      if (half == 0)
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float* ph = pb + size_t(h) * kAttnRows * p.nc_pad;
-        ph[size_t(t) * p.nc_pad + c] = acc[h];
-        if (t == 0) {
-          ph[size_t(128) * p.nc_pad + c] = s_m[h];
-          ph[size_t(129) * p.nc_pad + c] = s_l[h];
+        for (int h = 0; h < G; ++h) {
+          float* ph = pb + size_t(h) * kAttnRows * p.nc_pad;
+          ph[size_t(dd) * p.nc_pad + c] = acc[h];
+          if (dd == 0) {
+            ph[size_t(128) * p.nc_pad + c] = s_m[h];
+            ph[size_t(129) * p.nc_pad + c] = s_l[h];
+          }
         }
-      }
       __threadfence();
       __syncthreads();
       if (t == 0) {
@@ -624,6 +651,7 @@ decode_attn_kernel(DecAttnParams p) {
           s_den[t] = den;
         }
         __syncthreads();
+        if (half == 0) {
         float num[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) num[h] = 0.f;
@@ -633,7 +661,7 @@ decode_attn_kernel(DecAttnParams p) {
 #pragma unroll
           for (int h = 0; h < G; ++h)
             v[h] = __ldcg(reinterpret_cast<const float4*>(
-                pb + (size_t(h) * kAttnRows + t) * p.nc_pad + c4));
+                pb + (size_t(h) * kAttnRows + dd) * p.nc_pad + c4));
 #pragma unroll
           for (int h = 0; h < G; ++h) {
             const float* wv = s_w + h * p.nc_pad + c4;
@@ -644,7 +672,8 @@ decode_attn_kernel(DecAttnParams p) {
           }
         }
 #pragma unroll
-        for (int h = 0; h < G; ++h) ob[h * 128 + t] = __float2bfloat16_rn(num[h] / s_den[h]);
+        for (int h = 0; h < G; ++h) ob[h * 128 + dd] = __float2bfloat16_rn(num[h] / s_den[h]);
+        }
       }
     }
     __syncthreads();  // shared buffers are reused by the next item
@@ -693,7 +722,8 @@ DecSched dec_gemm_sched(int64_t rows, int64_t K, int B, int R) {
   uint32_t tcols = 32;
   while (tcols < static_cast<uint32_t>(s.NB * R)) tcols <<= 1;
   const int resident = (s.smem <= 113 * 1024 && 2 * tcols <= 512) ? 2 : 1;
-  // about `resident` CTAs per SM, one wave; fewer splits when the fp32
+  // about `resident` CTAs per SM, one wave (measured faster than one CTA per
+  // SM with room for the next kernel's CTA); fewer splits when the fp32
   // partials (written once, read once) would rival the weight bytes
   int splits = resident * sm_count() / (s.tiles > 0 ? s.tiles : 1);
   const int64_t by_traffic = K / (8 * int64_t(B));
