@@ -442,8 +442,6 @@ int run_decode_layer(const q3vl_config& c, const q3vl_layer& w, void* x, int32_t
   float* inv = reinterpret_cast<float*>(ws + L.inv);
   float* rowsq_h = reinterpret_cast<float*>(ws + L.rowsq_h);
   float* rowsq_x = reinterpret_cast<float*>(ws + L.rowsq_x);
-  float* part = reinterpret_cast<float*>(ws + L.part);
-  uint32_t* tickets = reinterpret_cast<uint32_t*>(ws + L.tickets);
   void* q = ws + L.q;
   void* o = ws + L.o;
   void* h = ws + L.h;
@@ -451,7 +449,7 @@ int run_decode_layer(const q3vl_config& c, const q3vl_layer& w, void* x, int32_t
   if (!x_stats_ready) Q3VL_CUDA(launch_rowstat(c, x, B, H, inv, st), "decode input rms");
 
   DecGemmArgs a{};
-  a.B = B; a.part = part; a.tickets = tickets; a.eps = static_cast<float>(c.rms_eps);
+  a.B = B; a.eps = static_cast<float>(c.rms_eps);
   a.n_heads = c.n_heads; a.n_kv = c.n_kv_heads;
   // P3+P4, with this token's K/V row written into the cache
   a.W = w.w_qkv; a.rows = qkv_dim(c); a.K = H; a.X = x;
@@ -470,20 +468,20 @@ int run_decode_layer(const q3vl_config& c, const q3vl_layer& w, void* x, int32_t
             "decode attention");
   // P6 (+ the row sums of squares of h for P7)
   DecGemmArgs r{};
-  r.B = B; r.part = part; r.tickets = tickets; r.eps = a.eps;
+  r.B = B; r.eps = a.eps;
   r.W = w.w_o; r.rows = H; r.K = Dq; r.X = o;
   r.N = H; r.out = h; r.resid = x; r.rowsq_out = rowsq_h;
   Q3VL_CUDA(launch_decode_gemm(Epi::kResidual, r, st), "decode o projection");
   // P7+P8
   DecGemmArgs g{};
-  g.B = B; g.part = part; g.tickets = tickets; g.eps = a.eps;
+  g.B = B; g.eps = a.eps;
   g.W = w.w_gu; g.rows = 2 * I; g.K = H; g.X = h;
   g.N = I; g.out = act; g.rowsq_in = rowsq_h;
   g.rowsq_n = static_cast<int>(H / 128); g.rowsq_width = static_cast<float>(H);
   Q3VL_CUDA(launch_decode_gemm(Epi::kSwiGLU, g, st), "decode gate/up projection");
   // P9 (+ the row sums of squares of x' for the next layer)
   DecGemmArgs d{};
-  d.B = B; d.part = part; d.tickets = tickets; d.eps = a.eps;
+  d.B = B; d.eps = a.eps;
   d.W = w.w_down; d.rows = H; d.K = I; d.X = act;
   d.N = H; d.out = x; d.resid = h; d.rowsq_out = leave_x_stats ? rowsq_x : nullptr;
   Q3VL_CUDA(launch_decode_gemm(Epi::kResidual, d, st), "decode down projection");
@@ -493,7 +491,8 @@ int run_decode_layer(const q3vl_config& c, const q3vl_layer& w, void* x, int32_t
 // Positions' cos/sin and zero tickets: once per decode call.
 int prepare_decode(const q3vl_config& c, const int32_t* pos, int32_t B, char* ws,
                    const DecLayout& L, cudaStream_t st) {
-  Q3VL_CUDA(cudaMemsetAsync(ws + L.tickets, 0, L.total - L.tickets, st), "clear decode tickets");
+  Q3VL_CUDA(cudaMemsetAsync(ws + L.att_tickets, 0, L.total - L.att_tickets, st),
+            "clear decode tickets");
   return cuda_check(launch_rope_table(c, pos, B, reinterpret_cast<float*>(ws + L.cos_sin), st),
                     "decode rope table");
 }

@@ -17,10 +17,12 @@
 // packed rows interleave 128 gate and 128 up rows) and the tokens are its N
 // operand (B rounded up to 16; TMA fills the missing rows with zeros), so
 // one 128 x NB x 64 MMA consumes one 16 KB weight box. The K range of each
-// row tile is split over several CTAs so that about two CTAs per SM stream
-// weights; each CTA stores its fp32 partial tile and the last CTA of a row
-// tile (a ticket counter) sums the partials in split order and runs the
-// epilogue of the prefill's step: 1/rms, bias, per-head RMSNorm and MRoPE
+// row tile is split over up to 8 CTAs (about two CTAs per SM stream
+// weights) that form one thread-block cluster: each CTA leaves its fp32
+// partial tile in its shared memory, and after a cluster barrier the CTAs
+// share out the tokens, each summing the partials of its tokens over DSMEM
+// in split order and running the epilogue of the prefill's step: 1/rms,
+// bias, per-head RMSNorm and MRoPE
 // with the K/V rows written into the cache (QKV); residual add and the row
 // sum of squares for the next norm (o-projection, down); SiLU(g) * u
 // (gate/up). The weights of a projection do not depend on the previous
@@ -36,18 +38,13 @@ namespace {
 constexpr int kDecThreads = 192;     // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr int kDecMaxB = 256;
 constexpr int kBK = 64;              // K elements per stage (one 128-byte row)
-
-__device__ __forceinline__ void dec_epi_sync() {
-  asm volatile("barrier.sync 1, 128;" ::: "memory");
-}
+constexpr int kDecMaxSplits = 8;     // portable cluster size
 
 __device__ __forceinline__ float bf16_to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
 
 struct DecGemmParams {
   int B, NB, R;          // tokens, MMA N (B rounded up to 16), 128-row blocks per tile
-  int n_k, splits, stages;
-  float* part;           // [tiles][splits][B][128 R] fp32 partial tiles
-  uint32_t* tickets;     // [tiles], zero between launches (the last CTA resets)
+  int n_k, splits, stages;  // splits = cluster size (<= kDecMaxSplits)
   int32_t* err;
   // epilogue
   int64_t N;             // output columns (kQkv: q columns nh*128; kSwiGLU: I)
@@ -179,7 +176,6 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
   uint64_t* acc_full = empty + S;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tile = static_cast<int>(blockIdx.x) / p.splits;
@@ -266,109 +262,72 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     }
     __syncwarp();
   } else {
-    // epilogue warps: TMEM lanes 32 q .. 32 q + 31 are weight rows (features)
+    // epilogue warps: wait for the accumulator (TMEM lanes 32 q .. 32 q + 31
+    // of warp q = warp % 4 are this tile's weight rows, columns are tokens)
     griddep_wait();
-    const int q = warp & 3;
-    const int e = warp - 2;  // 0..3
     bool ok = true;
     if (lane == 0) ok = mbar_wait(acc_full, 0, p.err, kWhereDecodeEpilogue, abort_flag);
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
     if (!ok) *abort_flag = 1;
-    dec_epi_sync();
-    const bool run = *abort_flag == 0;
-    tc_fence_after();
-    const uint32_t tbase = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
-    float* mine = p.part + (size_t(tile) * p.splits + split) * size_t(p.B) * (128 * R);
-    if (run) {
+  }
+  // Split sum over the cluster: the splits of a row tile are one cluster.
+  // Each CTA leaves its fp32 partial tile in its own (drained) stage ring;
+  // after a cluster barrier CTA `split` finishes tokens j = split (mod
+  // splits), reading every CTA's partial over DSMEM in split order. Every
+  // thread of every CTA of the cluster passes the same cluster barriers.
+  __syncthreads();  // all roles done: loads landed, MMAs committed or abandoned
+  const bool run = *abort_flag == 0;
+  tc_fence_after();
+  float* red = reinterpret_cast<float*>(smem);
+  const size_t ring = size_t(S) * (kABytes + b_bytes);
+  int chunk = static_cast<int>(ring / (512u * R)) / 16 * 16;  // tokens per round
+  if (chunk > p.NB) chunk = p.NB;
+  const int rstride = 128 * R;
 #pragma unroll 1
-      for (int r = 0; r < R; ++r) {
+  for (int j0 = 0; j0 < p.B; j0 += chunk) {
+    const int nj = p.B - j0 < chunk ? p.B - j0 : chunk;
+    if (warp >= 2 && run) {
+      const int q = warp & 3;
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
 #pragma unroll 1
-        for (int c0 = 0; c0 < p.NB; c0 += 16) {
+      for (int r = 0; r < R; ++r)
+#pragma unroll 1
+        for (int c0 = 0; c0 < nj; c0 += 16) {
           uint32_t u[16];
-          tmem_ld16(tbase + r * p.NB + c0, u);
+          tmem_ld16(tb + r * p.NB + j0 + c0, u);
           tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const int j = c0 + c;
-            if (j < p.B) mine[size_t(j) * (128 * R) + r * 128 + 32 * q + lane] = __uint_as_float(u[c]);
+          for (int c = 0; c < 16; ++c)
+            if (c0 + c < nj) red[(c0 + c) * rstride + r * 128 + 32 * q + lane] = __uint_as_float(u[c]);
+        }
+    }
+    cluster_sync();  // every CTA's partials of this round are in its shared memory
+    if (warp >= 2 && run) {
+      const int e = warp - 2;
+#pragma unroll 1
+      for (int jj = split + e * p.splits; jj < nj; jj += 4 * p.splits) {
+        float v[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        const uint32_t own = smem_u32(red + jj * rstride + lane);
+#pragma unroll
+        for (int sp = 0; sp < kDecMaxSplits; ++sp) {
+          if (sp < p.splits) {
+            const uint32_t ra = map_to_cta(own, static_cast<uint32_t>(sp));
+            float w[2][4];
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                w[r][i] = r < R ? ld_dsmem_f32(ra + 4u * (r * 128 + 32 * i)) : 0.f;
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+              for (int i = 0; i < 4; ++i) v[r][i] += w[r][i];
           }
         }
-      }
-      __threadfence();
-    }
-    tc_fence_before();
-    dec_epi_sync();
-    if (threadIdx.x == 64) {
-      // one thread decides for the four warps (the barriers below need all four)
-      bool last = false;
-      if (run) {
-        const uint32_t t = atomicAdd(p.tickets + tile, 1u);
-        last = t == static_cast<uint32_t>(p.splits - 1);
-        if (last) p.tickets[tile] = 0;  // every split has arrived: ready for the next launch
-      }
-      *last_flag = last ? 1 : 0;
-    }
-    dec_epi_sync();
-    if (*last_flag) {
-      __threadfence();
-      // Sum the splits in split order into shared memory (the drained stage
-      // ring), all 128 threads with up to 16 independent 16-byte loads in
-      // flight each, then run the epilogue one token per warp from there.
-      const float4* base4 = reinterpret_cast<const float4*>(
-          p.part + size_t(tile) * p.splits * size_t(p.B) * (128 * R));
-      float4* red = reinterpret_cast<float4*>(smem);
-      const size_t ring = size_t(S) * (kABytes + b_bytes);
-      const int chunk = static_cast<int>(ring / (512u * R)) < p.B
-                            ? static_cast<int>(ring / (512u * R)) : p.B;
-      const size_t stride4 = size_t(p.B) * (32 * R);  // float4 per split
-      const int et = threadIdx.x - 64;
-#pragma unroll 1
-      for (int j0 = 0; j0 < p.B; j0 += chunk) {
-        const int nj = p.B - j0 < chunk ? p.B - j0 : chunk;
-        const int n4 = nj * 32 * R;
-        const float4* src = base4 + size_t(j0) * (32 * R);
-#pragma unroll 1
-        for (int q0 = et; q0 < n4; q0 += 4 * 128) {
-          float4 acc[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 1
-          for (int s0 = 0; s0 < p.splits; s0 += 4) {
-            float4 v[4][4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-#pragma unroll
-              for (int k = 0; k < 4; ++k)
-                v[u][k] = (s0 + k < p.splits && q0 + 128 * u < n4)
-                              ? __ldcg(src + size_t(s0 + k) * stride4 + q0 + 128 * u)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                acc[u].x += v[u][k].x; acc[u].y += v[u][k].y;
-                acc[u].z += v[u][k].z; acc[u].w += v[u][k].w;
-              }
-          }
-#pragma unroll
-          for (int u = 0; u < 4; ++u)
-            if (q0 + 128 * u < n4) red[q0 + 128 * u] = acc[u];
-        }
-        dec_epi_sync();
-        const float* redf = reinterpret_cast<const float*>(red);
-#pragma unroll 1
-        for (int j = e; j < nj; j += 4) {
-          float v[2][4];
-#pragma unroll
-          for (int r = 0; r < 2; ++r)
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              v[r][i] = r < R ? redf[size_t(j) * (128 * R) + r * 128 + lane + 32 * i] : 0.f;
-          dec_epilogue_token<EPI>(p, tile, j0 + j, lane, v);
-        }
-        dec_epi_sync();
+        dec_epilogue_token<EPI>(p, tile, j0 + jj, lane, v);
       }
     }
+    cluster_sync();  // no CTA overwrites or leaves its buffer while another may read it
   }
   tc_fence_before();
   __syncthreads();
@@ -723,11 +682,10 @@ DecSched dec_gemm_sched(int64_t rows, int64_t K, int B, int R) {
   while (tcols < static_cast<uint32_t>(s.NB * R)) tcols <<= 1;
   const int resident = (s.smem <= 113 * 1024 && 2 * tcols <= 512) ? 2 : 1;
   // about `resident` CTAs per SM, one wave (measured faster than one CTA per
-  // SM with room for the next kernel's CTA); fewer splits when the fp32
-  // partials (written once, read once) would rival the weight bytes
+  // SM with room for the next kernel's CTA); the splits of a tile form one
+  // cluster, at most the portable cluster size
   int splits = resident * sm_count() / (s.tiles > 0 ? s.tiles : 1);
-  const int64_t by_traffic = K / (8 * int64_t(B));
-  if (splits > by_traffic) splits = static_cast<int>(by_traffic);
+  if (splits > kDecMaxSplits) splits = kDecMaxSplits;
   if (splits > s.n_k) splits = s.n_k;
   s.splits = splits < 1 ? 1 : splits;
   return s;
@@ -750,22 +708,11 @@ DecLayout dec_layout(const q3vl_config& c, int B, int64_t cap) {
   L.o = take(size_t(B) * Dq * 2);
   L.h = take(size_t(B) * H * 2);
   L.act = take(size_t(B) * I * 2);
-  const DecSched sc[4] = {dec_gemm_sched(qkv_dim(c), H, B, 1), dec_gemm_sched(H, Dq, B, 1),
-                          dec_gemm_sched(2 * I, H, B, 2), dec_gemm_sched(H, I, B, 1)};
-  size_t part = 0;
-  int tiles = 0;
-  for (const DecSched& s : sc) {
-    const size_t b = size_t(s.tiles) * s.splits * B * 128 * s.R * sizeof(float);
-    if (b > part) part = b;
-    if (s.tiles > tiles) tiles = s.tiles;
-  }
-  L.part = take(part);
   const int G = c.n_heads / c.n_kv_heads;
   const int64_t nc_pad = ((cap + kAttnCH - 1) / kAttnCH + 3) / 4 * 4;
   L.att_items = int64_t(B) * c.n_kv_heads * ((cap + kAttnCH - 1) / kAttnCH);
   L.att_part = take(size_t(B) * c.n_kv_heads * G * kAttnRows * nc_pad * sizeof(float));
-  // the two ticket regions come last, so one memset clears both
-  L.tickets = take(size_t(tiles) * sizeof(uint32_t));
+  // the ticket region comes last; each decode call clears it once
   L.att_tickets = take(size_t(B) * c.n_kv_heads * sizeof(uint32_t));
   L.total = off;
   return L;
@@ -773,19 +720,29 @@ DecLayout dec_layout(const q3vl_config& c, int B, int64_t cap) {
 
 namespace {
 
+// Launch as a programmatic dependent of the previous kernel in the stream,
+// optionally in clusters of `cluster_x` CTAs along x.
 template <typename K, typename... Args>
 cudaError_t launch_pdl(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                       Args... args) {
+                       int cluster_x, Args... args) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   at[0].val.programmaticStreamSerializationAllowed = 1;
+  int n = 1;
+  if (cluster_x > 1) {
+    at[1].id = cudaLaunchAttributeClusterDimension;
+    at[1].val.clusterDim.x = static_cast<unsigned>(cluster_x);
+    at[1].val.clusterDim.y = 1;
+    at[1].val.clusterDim.z = 1;
+    n = 2;
+  }
   cfg.attrs = at;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = n;
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
@@ -806,7 +763,7 @@ cudaError_t launch_dec_epi(const DecGemmArgs& a, int R, cudaStream_t st) {
   DecGemmParams p{};
   p.B = a.B; p.NB = s.NB; p.R = R;
   p.n_k = s.n_k; p.splits = s.splits; p.stages = s.stages;
-  p.part = a.part; p.tickets = a.tickets; p.err = device_error_ptr();
+  p.err = device_error_ptr();
   p.N = a.N; p.out = static_cast<__nv_bfloat16*>(a.out);
   p.resid = static_cast<const __nv_bfloat16*>(a.resid);
   p.rowsq_out = a.rowsq_out; p.rowsq_in = a.rowsq_in; p.rowsq_n = a.rowsq_n;
@@ -818,7 +775,7 @@ cudaError_t launch_dec_epi(const DecGemmArgs& a, int R, cudaStream_t st) {
   p.v_cache = static_cast<__nv_bfloat16*>(a.v_cache);
   p.cap = a.cap; p.n_seq = a.n_seq; p.seq = a.seq; p.len = a.len;
   const cudaError_t e = launch_pdl(decode_gemm_kernel<EPI>, dim3(s.tiles * s.splits),
-                                   dim3(kDecThreads), s.smem, st, tmW, tmX, p);
+                                   dim3(kDecThreads), s.smem, st, s.splits, tmW, tmX, p);
   if (e != cudaSuccess) return e;
   return counted_launch(1);
 }
@@ -834,7 +791,7 @@ cudaError_t launch_attn_g(const DecAttnParams& p, int grid, cudaStream_t st) {
     smem_set = smem;
   }
   const cudaError_t e =
-      launch_pdl(decode_attn_kernel<G>, dim3(grid), dim3(kAttnThreads), smem, st, p);
+      launch_pdl(decode_attn_kernel<G>, dim3(grid), dim3(kAttnThreads), smem, st, 1, p);
   if (e != cudaSuccess) return e;
   return counted_launch(1);
 }

@@ -144,9 +144,7 @@ struct DecLayout {
   size_t o = 0;         // bf16 [B][Dq]
   size_t h = 0;         // bf16 [B][H]
   size_t act = 0;       // bf16 [B][I]
-  size_t part = 0;      // fp32 partial tiles of the split projections
   size_t att_part = 0;  // fp32 [att_items][G][132] attention chunk partials
-  size_t tickets = 0;   // uint32 [max tiles], zero between launches
   size_t att_tickets = 0;  // uint32 [B][nkv], zero between launches
   int64_t att_items = 0;
   size_t total = 0;
@@ -158,8 +156,6 @@ struct DecGemmArgs {
   int64_t rows, K;
   const void* X;        // bf16 [B, K] tokens
   int B;
-  float* part;
-  uint32_t* tickets;
   int64_t N;            // output row stride / columns
   void* out;
   const void* resid;
