@@ -687,6 +687,11 @@ DecSched dec_gemm_sched(int64_t rows, int64_t K, int B, int R) {
   int splits = resident * sm_count() / (s.tiles > 0 ? s.tiles : 1);
   if (splits > kDecMaxSplits) splits = kDecMaxSplits;
   if (splits > s.n_k) splits = s.n_k;
+  // A cluster must fit inside one GPC. Counting each GPC as 16 SMs (a
+  // B200 has 8 GPCs of 148 SMs in all), lower the split count until every
+  // row tile's cluster is resident in the first wave.
+  const int gpcs = sm_count() / 18 > 1 ? sm_count() / 18 : 1;
+  while (splits > 1 && (16 * resident / splits) * gpcs < s.tiles) --splits;
   s.splits = splits < 1 ? 1 : splits;
   return s;
 }
