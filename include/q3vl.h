@@ -266,8 +266,8 @@ int q3vl_final_norm(const q3vl_config* cfg, void* x, int64_t S, const void* gain
 typedef struct q3vl_kv_cache {
   void* k;        /* device bf16 [n_seq][cap][nkv*hd], 16-byte aligned */
   void* v;        /* device bf16 [n_seq][cap][nkv*hd], 16-byte aligned */
-  int64_t cap;    /* rows per sequence slot, >= 1 */
-  int32_t n_seq;  /* sequence slots, >= 1 */
+  int64_t cap;    /* rows per sequence slot, 1 <= cap <= 131072 */
+  int32_t n_seq;  /* sequence slots, >= 1, with n_seq * cap < 2^31 */
 } q3vl_kv_cache;
 
 /* q3vl_layer_prefill / q3vl_stack_prefill that also write rows 0..S-1 of

@@ -400,6 +400,10 @@ int check_kv(const q3vl_config& c, const q3vl_kv_cache* kv, const char* what) {
   Q3VL_TRY(check_ptr(kv->v, "kv cache v"));
   if (kv->cap < 1 || kv->n_seq < 1)
     return set_error(Q3VL_EINVAL, "kv cache needs cap >= 1 and n_seq >= 1");
+  if (kv->cap > 131072)
+    return set_error(Q3VL_EUNSUPPORTED, "kv cache cap above 131072 rows per slot");
+  if (int64_t(kv->n_seq) * kv->cap > int64_t(0x7fffffff))
+    return set_error(Q3VL_EINVAL, "kv cache n_seq * cap must stay below 2^31 rows");
   (void)c;
   return Q3VL_OK;
 }

@@ -166,6 +166,8 @@ def test_decode_argument_checks(lib):
     assert dec(B=257) == -1
     assert dec(ws_bytes=1024) == -5
     assert dec(kv_=_kv(cap=0)) == -1
+    assert dec(kv_=_kv(cap=131073)) == -8
+    assert dec(kv_=_kv(cap=131072, n_seq=1 << 15)) == -1
     assert dec(cfg=_cfg(dtype="fp32")) == -8
     assert lib.q3vl_decode_advance(0, P, P, None) == -1
     # prefill into a cache: S above the capacity, or a slot outside [0, n_seq)
