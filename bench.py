@@ -60,6 +60,12 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true",
                     help="skip the one-token decode measurement of the 36-layer stack")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="run only the decode measurement and print its JSON (for profiling)")
+    ap.add_argument("--decode-batches", default="1,32",
+                    help="comma-separated decode batch sizes")
+    ap.add_argument("--decode-layers", type=int, default=36,
+                    help="layers of the decode stack (36 = the 4B shape)")
     return ap.parse_args()
 
 
@@ -414,6 +420,14 @@ def main():
     if args.impl == "reference":
         reference_arm(args, w)
         return
+    if args.decode_only:
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        batches = tuple(int(b) for b in args.decode_batches.split(","))
+        out = decode_leg(dev, args.steps, max(3, args.warmup), batches,
+                         syn.Q4B_DECODE.with_layers(args.decode_layers))
+        print(json.dumps(out), flush=True)
+        return
     rank, world, local = dist_setup(args.gpus)
     if world > 1:
         import datetime
@@ -482,7 +496,9 @@ def main():
 
     decode = None
     if world == 1 and not args.no_decode:
-        decode = decode_leg(dev, min(args.steps, 400), max(3, min(args.warmup, 20)))
+        decode = decode_leg(dev, min(args.steps, 400), max(3, min(args.warmup, 20)),
+                            tuple(int(b) for b in args.decode_batches.split(",")),
+                            syn.Q4B_DECODE.with_layers(args.decode_layers))
 
     burst, sustained, hbm, src = peaks()
     gemm_f, attn_f = layer_flops(w)
