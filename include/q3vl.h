@@ -53,7 +53,7 @@ enum q3vl_status_code {
   Q3VL_EWORKSPACE = -5,   /* workspace or packed buffer too small */
   Q3VL_ECUDA = -6,        /* a CUDA runtime call failed */
   Q3VL_ETIMEOUT = -7,     /* a device-side wait hit its time limit */
-  Q3VL_EUNSUPPORTED = -8  /* head_dim != 128, video grid (t > 1), ... */
+  Q3VL_EUNSUPPORTED = -8  /* head_dim != 128, a decode shape outside its limits, ... */
 };
 
 enum q3vl_dtype { Q3VL_DTYPE_FP32 = 0, Q3VL_DTYPE_BF16 = 1 };
@@ -120,15 +120,18 @@ int q3vl_layer_views(const q3vl_config* cfg, const void* packed, q3vl_layer* out
  * P0. MRoPE position ids ([P] `mrope_positions`, [C] `mrope_positions`).
  * token_types: device uint8 [S], 0 = text, 1 = image placeholder.
  * grids:       device int32 [n_grids][3] = (t, merged rows, merged cols) of
- *              each image in prompt order; t must be 1.
+ *              each image or video in prompt order; t = frames (1 for a
+ *              still image), all three >= 1.
  * pos:         device int32 [3][S] out, axis-major (t row, h row, w row).
- * info:        device int32 [2] out: info[0] = status (Q3VL_OK, Q3VL_EGRID
- *              or Q3VL_EUNSUPPORTED), info[1] = next position (one past the
- *              largest position on any axis).
- * A text token takes (c, c, c) and advances c by 1; image g's k-th token
- * takes (c, c + k / cols, c + k % cols) and the image advances c by
- * max(rows, cols). Grids are consumed whole and in order. 1 <= S <= 2^30,
- * 0 <= n_grids <= 4096; otherwise Q3VL_EINVAL. Bit-exact integer work.
+ * info:        device int32 [2] out: info[0] = status (Q3VL_OK or
+ *              Q3VL_EGRID), info[1] = next position (one past the largest
+ *              position on any axis).
+ * A text token takes (c, c, c) and advances c by 1. Grid g occupies
+ * t * rows * cols placeholder tokens in (frame, row, col) order; token
+ * (f, r, q) takes (c + f, c + r, c + q), and the grid advances c by
+ * max(rows, cols) only ([P] `mrope_positions`). Grids are consumed whole and
+ * in order. 1 <= S <= 2^30, 0 <= n_grids <= 4096; otherwise Q3VL_EINVAL.
+ * Bit-exact integer work.
  * ------------------------------------------------------------------------- */
 int q3vl_mrope_positions(const uint8_t* token_types, int64_t S, const int32_t* grids,
                          int32_t n_grids, int32_t* pos, int32_t* info, q3vl_stream stream);

@@ -56,11 +56,14 @@ def mrope_positions_tokens(token_types: Sequence[int],
 
     inferencelayer ``vision.rs``, ``mrope_positions``: a text token takes
     (cur, cur, cur) and advances cur by one. An image placeholder starts the
-    next grid (t, rows, cols) of merged tokens; its k-th token takes
-    (cur, cur + k div cols, cur + k mod cols) (row-major 'ij' order), and the
-    whole image advances cur by max(rows, cols), not by its token count.
-    Grids are consumed whole and in order, so two adjacent images need no
-    text between them. ``next`` is one past the largest position on any axis.
+    next grid (t, rows, cols) of merged tokens, t frames of rows x cols (t = 1
+    for a still image); its tokens follow the meshgrid of (frame, row, col) in
+    'ij' order, token (f, r, c) taking (cur + f, cur + r, cur + c), and the
+    whole grid advances cur by max(rows, cols) -- neither its token count nor
+    its frame count. Grids are consumed whole and in order, so two adjacent
+    images need no text between them. ``next`` is one past the largest
+    position on any axis (with t > max(rows, cols) frames that is on the t
+    axis, beyond where the following text resumes).
 
     Returns (pos int64 [3, S], next).
     """
@@ -79,15 +82,17 @@ def mrope_positions_tokens(token_types: Sequence[int],
             raise OracleError("more image placeholders than grids")
         t, rows, cols = grids[gi]
         gi += 1
-        if t != 1:
-            raise OracleError("only still images (grid t == 1) are supported")
-        n = rows * cols
+        if t < 1 or rows < 1 or cols < 1:
+            raise OracleError("grid sizes must be >= 1")
+        n = t * rows * cols
         if i + n > S or any(token_types[j] != 1 for j in range(i, i + n)):
             raise OracleError("image placeholder run shorter than its grid")
-        for k in range(n):
-            pos[0, i + k] = cur
-            pos[1, i + k] = cur + k // cols
-            pos[2, i + k] = cur + k % cols
+        k = 0
+        for f in range(t):
+            for r in range(rows):
+                for c in range(cols):
+                    pos[:, i + k] = (cur + f, cur + r, cur + c)
+                    k += 1
         cur += max(rows, cols)
         i += n
     if gi != len(grids):

@@ -35,7 +35,8 @@ int32_t* device_error_ptr() {
 // One block walks the prompt in chunks. With c(i) = number of image tokens
 // before token i, a text token's counter is (i - c) plus the advances of
 // the grids completed before it; image token i belongs to grid g with
-// gstart[g] <= c < gstart[g+1] and sits at k = c - gstart[g] in it.
+// gstart[g] <= c < gstart[g+1] and sits at k = c - gstart[g] in it, i.e. at
+// frame k / (rows cols), row (k mod rows cols) / cols, column k mod cols.
 // ---------------------------------------------------------------------------
 constexpr int kMaxGrids = 4096;
 constexpr int kPosThreads = 1024;
@@ -62,11 +63,10 @@ positions_kernel(const uint8_t* __restrict__ tt, int64_t S, const int32_t* __res
   __syncthreads();  // the status word is cleared before any check can fail
   for (int g = tid; g < n_grids; g += kPosThreads) {
     const int t = grids[3 * g], r = grids[3 * g + 1], c = grids[3 * g + 2];
-    if (t != 1) pos_fail(info, Q3VL_EUNSUPPORTED);
-    const bool ok = r >= 1 && c >= 1 && int64_t(r) * c <= S;
+    const bool ok = t >= 1 && r >= 1 && c >= 1 && int64_t(t) * r * c <= S;
     if (!ok) pos_fail(info, Q3VL_EGRID);
-    gstart[g + 1] = ok ? r * c : 0;
-    gadv[g + 1] = ok ? max(r, c) : 0;
+    gstart[g + 1] = ok ? t * r * c : 0;  // t frames of r x c tokens
+    gadv[g + 1] = ok ? max(r, c) : 0;    // the counter moves by the longer side only
   }
   __syncthreads();
   if (tid == 0) {
@@ -143,12 +143,13 @@ positions_kernel(const uint8_t* __restrict__ tt, int64_t S, const int32_t* __res
         const int g = lo;
         const int32_t k = c - gstart[g];
         if (k > 0 && tt[i - 1] != 1) pos_fail(info, Q3VL_EGRID);  // run broken by text
-        const int32_t cols = max(grids[3 * g + 2], 1);
+        const int32_t rows = max(grids[3 * g + 1], 1), cols = max(grids[3 * g + 2], 1);
+        const int32_t frame = k / (rows * cols), rem = k % (rows * cols);
         const int32_t b = static_cast<int32_t>(i - k) - gstart[g] + gadv[g];
-        p0 = b;
-        p1 = b + k / cols;
-        p2 = b + k % cols;
-        my_max = max(my_max, max(p1, p2));
+        p0 = b + frame;
+        p1 = b + rem / cols;
+        p2 = b + rem % cols;
+        my_max = max(my_max, max(p0, max(p1, p2)));
         ++c;
       }
       pos[i] = p0;

@@ -102,3 +102,24 @@ def test_timeout_selftest_recovers():
     w = syn.TINY_FP32.with_seq(16)
     xin, got, ref = run_layer(w)
     check(w, xin, got, ref)
+
+
+def test_layer_with_a_video_span():
+    # a prompt holding a 3-frame video: the t axis varies inside the span
+    # (inferencelayer vision.rs `mrope_positions`), so the t slots of MRoPE
+    # rotate differently per frame
+    m = q3()
+    w = syn.Q2B_LAYER.with_seq(900)
+    cfg = m.config_of(w)
+    types = [0] * 100 + [1] * (3 * 10 * 12) + [0] * (900 - 100 - 360)
+    grids = [(3, 10, 12)]
+    pos, nxt = m.mrope_positions(torch.tensor(types, dtype=torch.uint8, device="cuda"),
+                                 torch.tensor(grids, dtype=torch.int32, device="cuda"))
+    ref_pos, ref_next = O.mrope_positions_tokens(types, grids)
+    assert np.array_equal(pos.cpu().numpy(), ref_pos) and nxt == ref_next
+    raw, packed = layer_on_device(w)
+    x = syn.hidden_input(w)
+    xd = x.cuda().clone()
+    m.layer_prefill(cfg, packed, xd, pos)
+    m.check_device()
+    check(w, host(x), host(xd), O.layer(O.Config.of(w), raw, x, ref_pos))

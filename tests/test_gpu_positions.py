@@ -56,12 +56,31 @@ def test_random_prompts_long():
     ([0, 1, 1, 1], [], -3),
     ([0, 0], [(1, 1, 1)], -3),
     ([1, 1, 0, 1, 1], [(1, 2, 2)], -3),
-    ([1, 1], [(2, 1, 1), (1, 1, 1)], -8),
+    ([1, 1], [(2, 1, 1), (1, 1, 1)], -3),   # the 2-frame video takes both tokens
+    ([1], [(0, 1, 1)], -3),                 # a grid with no frames
 ])
 def test_mismatch_reported(types, grids, code):
     with pytest.raises(q3().Q3VLError) as e:
         _run(types, grids)
     assert e.value.code == code
+
+
+def test_random_prompts_with_videos():
+    # videos (t frames) mixed with still images and text, several scan chunks
+    rng = np.random.default_rng(8)
+    for trial in range(12):
+        types, grids = [], []
+        while len(types) < 6000 + 700 * trial:
+            types += [0] * int(rng.integers(0, 30))
+            if rng.random() < 0.8:
+                t = int(rng.integers(1, 9)) if rng.random() < 0.5 else 1
+                r, c = int(rng.integers(1, 17)), int(rng.integers(1, 17))
+                types += [1] * (t * r * c)
+                grids.append((t, r, c))
+        pos, nxt = _run(types, grids)
+        ref, ref_next = O.mrope_positions_tokens(types, grids)
+        assert np.array_equal(pos.cpu().numpy(), ref)
+        assert nxt == ref_next
 
 
 def test_single_token():

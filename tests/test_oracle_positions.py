@@ -31,7 +31,27 @@ def _spans_from(types, grids):
 @pytest.mark.parametrize("name", all_position_files())
 def test_span_form_matches_token_form_on_golden(name):
     types, grids, want, _ = load_positions(name)
+    if any(g[0] != 1 for g in grids):
+        pytest.skip("the span form (cortiq qwen3te.rs) has no frame axis")
     assert mrope_positions_spans(len(types), _spans_from(types, grids)).tolist() == want
+
+
+def test_video_frames_shift_only_t_and_text_resumes_after_the_longer_side():
+    # inferencelayer vision.rs `mrope_positions`: frame f of a (t, h, w) grid
+    # is frame 0 shifted by f on the t axis alone; the counter moves by max(h, w)
+    rng = np.random.default_rng(11)
+    for _ in range(100):
+        t, r, c = (int(v) for v in rng.integers(1, 7, size=3))
+        lead = int(rng.integers(0, 5))
+        types = [0] * lead + [1] * (t * r * c) + [0] * 3
+        pos, nxt = mrope_positions_tokens(types, [(t, r, c)])
+        still, _ = mrope_positions_tokens([0] * lead + [1] * (r * c), [(1, r, c)])
+        for f in range(t):
+            blk = pos[:, lead + f * r * c: lead + (f + 1) * r * c]
+            assert (blk - still[:, lead:] == np.array([[f], [0], [0]])).all()
+        tail = pos[:, lead + t * r * c:]
+        assert (tail == lead + max(r, c) + np.arange(3)).all()
+        assert nxt == max(lead + t - 1, lead + max(r, c) + 2) + 1
 
 
 def test_text_only_is_arange():
@@ -86,7 +106,8 @@ def test_workload_4b_positions():
     ([0, 1, 1, 0], [(1, 1, 3)]),          # run shorter than its grid
     ([0, 1, 1, 1], []),                   # placeholders but no grid
     ([0, 0], [(1, 1, 1)]),                # grid left over
-    ([1, 1], [(2, 1, 1), (1, 1, 1)]),     # video grid (t > 1) is not supported
+    ([1, 1], [(2, 1, 1), (1, 1, 1)]),     # the 2-frame video takes both tokens: a grid is left
+    ([1], [(0, 1, 1)]),                   # a grid with no frames
 ])
 def test_rejects_mismatch(types, grids):
     with pytest.raises(OracleError):
