@@ -22,7 +22,9 @@ Sources (the pages' own items; the pages print Rust, restated here):
   before the q/k norm), the DeepStack contract and input validation of
   ``forward_text_prefill_logits_last``, and "Why no KV cache yet" (a decoded
   token is the last row of the prefill re-run over prompt + decoded tokens),
-  which defines the incremental decode at the end of this module.
+  which defines the incremental decode at the end of this module; and the
+  same function's step 1 (token embedding lookup and soft-token splice) and
+  step 4 (final norm and LM head, tied or untied).
 
 Parity status: every function here is pinned by the ``-m "not gpu"`` tests
 (hand-computed grids, closed forms, brute force, invariants). The composed
@@ -31,7 +33,8 @@ special cases (zero projections, uniform attention, one-hot FFN); the pages
 print no numeric output of a full layer, so that composition has no external
 numeric pin. The decode functions are pinned against that prefill layer
 (the last row of a re-run prefill) and against closed forms that hold for
-arbitrary cache contents.
+arbitrary cache contents. The embedding gather and LM head are pinned by
+closed forms (coded table rows, a scaled basis vector).
 """
 from __future__ import annotations
 
@@ -506,3 +509,52 @@ def stack_decode(cfg: Config, layers: List[Dict], x_new, pos_new: np.ndarray,
     if final_norm is not None:
         h = rms_norm(h, _np(final_norm, dtype), cfg.rms_eps)
     return h, new
+
+
+# ---------------------------------------------------------------------------
+# The steps either side of the layers: embedding gather with the soft-token
+# splice, and the final norm + LM head
+# ---------------------------------------------------------------------------
+
+def embed(table, tokens: Sequence[int], soft_rows: Sequence[int] = (), soft=None,
+          dtype=np.float64) -> np.ndarray:
+    """x[p] = table[tokens[p]], then x[soft_rows[k]] = soft[k] (the spliced rows).
+
+    hf2q ``qwen3vl_text/forward.rs``, ``forward_text_prefill_logits_last``,
+    step 1: the token embedding lookup, then every soft-token injection
+    overwrites its rows with the supplied embeddings. The injections must lie
+    inside the prompt and must not overlap; here they are given as one list of
+    destination rows with one embedding row each (a range [s, e) is the rows
+    s..e-1), so "overlap" is a repeated row. A token id outside the table is
+    an error as well.
+    """
+    table = _np(table, dtype)
+    tokens = np.asarray(tokens, dtype=np.int64)
+    S, vocab = len(tokens), table.shape[0]
+    if S == 0:
+        raise OracleError("empty token list")
+    if tokens.min() < 0 or tokens.max() >= vocab:
+        raise OracleError("token id outside the embedding table")
+    x = table[tokens].copy()
+    soft_rows = np.asarray(soft_rows, dtype=np.int64)
+    if len(soft_rows):
+        soft = _np(soft, dtype)
+        if soft.shape[0] != len(soft_rows):
+            raise OracleError("soft-token rows and embeddings disagree")
+        if soft_rows.min() < 0 or soft_rows.max() >= S:
+            raise OracleError("soft-token row outside the prompt")
+        if len(np.unique(soft_rows)) != len(soft_rows):
+            raise OracleError("soft-token rows overlap")
+        x[soft_rows] = soft
+    return x
+
+
+def lm_head(cfg: Config, x_rows, final_norm, weight, dtype=np.float64) -> np.ndarray:
+    """logits = RMSNorm(x, final_norm) W^T for each given row ([rows, vocab]).
+
+    hf2q ``qwen3vl_text/forward.rs``, step 4: the last position's residual
+    row goes through the final RMSNorm and the LM head; W is the output
+    weight, or the token embedding table itself when the embeddings are tied.
+    """
+    xn = rms_norm(_np(x_rows, dtype), _np(final_norm, dtype), cfg.rms_eps)
+    return xn @ _np(weight, dtype).T
