@@ -25,6 +25,7 @@ the data path. --impl reference times the CPU oracle itself on the host.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import os
@@ -408,6 +409,37 @@ def decode_leg(dev, steps, warmup, batches=(1, 32), w=None):
                                      "peak_source": f"{src} copy bandwidth"}}
         del graph
     del kvs, layers
+    torch.cuda.empty_cache()
+    # final norm + LM head of the decoded rows (tied: the embedding table is
+    # the head), Qwen3-VL's vocabulary; bytes = the [vocab, H] bf16 weight
+    vocab = 151936
+    gen = torch.Generator(device=dev).manual_seed(23)
+    table = (0.02 * torch.randn(vocab, w.hidden, generator=gen, device=dev)).to(torch.bfloat16)
+    gain = (1.0 + 0.1 * torch.randn(w.hidden, generator=gen, device=dev)).to(torch.bfloat16)
+    head = {}
+    for B in batches:
+        xr = torch.randn(B, w.hidden, generator=gen, device=dev).to(torch.bfloat16)
+        logits = torch.empty((B, vocab), dtype=torch.float32, device=dev)
+        hws = torch.empty(int(q3.lib().q3vl_lm_head_workspace_bytes(ctypes.byref(cfg), B)),
+                          dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            q3.lm_head(cfg, xr, gain, table, logits, hws)
+        n = 50
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(n):
+            q3.lm_head(cfg, xr, gain, table, logits, hws)
+        e1.record()
+        torch.cuda.synchronize()
+        q3.check_device()
+        t = e0.elapsed_time(e1) / 1e3 / n
+        head_bytes = vocab * w.hidden * 2 + B * (w.hidden * 4 + vocab * 4)
+        head[f"B{B}"] = {"us": 1e6 * t, "vocab": vocab,
+                         "roofline": {"bound": "hbm", "achieved": head_bytes / t / 1e9, "peak": hbm,
+                                      "unit": "GB/s", "frac": head_bytes / t / 1e9 / hbm}}
+    out["lm_head"] = head
+    del table
     torch.cuda.empty_cache()
     return out
 

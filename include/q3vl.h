@@ -324,6 +324,44 @@ int q3vl_stack_decode(const q3vl_config* cfg, int32_t n_layers, const q3vl_layer
 int q3vl_decode_advance(int32_t B, int32_t* pos, int32_t* len, q3vl_stream stream);
 
 /* ---------------------------------------------------------------------------
+ * The steps either side of the layers ([H] `forward_text_prefill_logits_last`
+ * steps 1 and 4).
+ * ------------------------------------------------------------------------- */
+
+/* Token embedding gather with the soft-token splice: x[p] = table[tokens[p]]
+ * for p < S, then x[soft_rows[k]] = soft[k] (the rows a vision tower's
+ * embeddings replace; an injected range [s, e) is the rows s..e-1).
+ * table:  device [vocab, H] in cfg dtype, 16-byte aligned.
+ * tokens: device int32 [S]. An id outside [0, vocab) is the device error
+ *         Q3VL_ERANGE, and that row is left zero.
+ * soft, soft_rows: device [n_soft, H] (cfg dtype) and int32 [n_soft], or NULL
+ *         with n_soft = 0. Rows outside [0, S) or repeated (overlapping
+ *         injections) are the device error Q3VL_ERANGE ([H] validation).
+ * x:      device [S, H] out.
+ * ws:     device scratch of >= 4*S bytes, 256-byte aligned, when n_soft > 0
+ *         (a row map); may be NULL otherwise. */
+int q3vl_embed(const q3vl_config* cfg, const void* table, int64_t vocab, const int32_t* tokens,
+               int64_t S, const void* soft, const int32_t* soft_rows, int32_t n_soft, void* x,
+               void* ws, size_t ws_bytes, q3vl_stream stream);
+
+/* Workspace bytes of q3vl_lm_head for B rows (0 for invalid arguments). */
+size_t q3vl_lm_head_workspace_bytes(const q3vl_config* cfg, int32_t B);
+
+/* Final norm and LM head: logits[b] = RMSNorm(x[b], final_norm) W^T in fp32
+ * (bf16 configs only; the rows are normalised in fp32 and rounded to bf16
+ * before the product).
+ * x:          device bf16 [B, H], 1 <= B <= 256: e.g. the last row of a
+ *             prefill, or the B decoded tokens.
+ * final_norm: device bf16 [H] gain, or NULL for rows already normalised.
+ * weight:     device bf16 [vocab, H], 16-byte aligned: the output weight, or
+ *             the token embedding table when the embeddings are tied.
+ * logits:     device fp32 [B, vocab] out.
+ * ws:         >= q3vl_lm_head_workspace_bytes(cfg, B) bytes, 256-byte aligned. */
+int q3vl_lm_head(const q3vl_config* cfg, const void* x, int32_t B, const void* final_norm,
+                 const void* weight, int64_t vocab, float* logits, void* ws, size_t ws_bytes,
+                 q3vl_stream stream);
+
+/* ---------------------------------------------------------------------------
  * Diagnostics.
  * ------------------------------------------------------------------------- */
 

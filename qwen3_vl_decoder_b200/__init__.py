@@ -285,6 +285,40 @@ def decode_advance(pos: torch.Tensor, lens: torch.Tensor, stream=None) -> None:
 
 
 # ---------------------------------------------------------------------------
+# Embedding gather (+ soft-token splice) and LM head
+# ---------------------------------------------------------------------------
+def embed(cfg: Config, table: torch.Tensor, tokens: torch.Tensor,
+          soft: Optional[torch.Tensor] = None, soft_rows: Optional[torch.Tensor] = None,
+          x: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """x[p] = table[tokens[p]], then x[soft_rows[k]] = soft[k]; returns x [S, H]."""
+    S = tokens.numel()
+    x = torch.empty((S, cfg.hidden), dtype=table.dtype, device=table.device) if x is None else x
+    n_soft = 0 if soft_rows is None else soft_rows.numel()
+    ws = torch.empty(max(1, 4 * S), dtype=torch.uint8, device=table.device) if n_soft else None
+    _check(lib().q3vl_embed(ctypes.byref(cfg), _ptr(table), table.shape[0], _ptr(tokens), S,
+                           _ptr(soft), _ptr(soft_rows), n_soft, _ptr(x), _ptr(ws),
+                           0 if ws is None else ws.numel(), _stream(stream)))
+    return x
+
+
+def lm_head(cfg: Config, x_rows: torch.Tensor, final_norm: Optional[torch.Tensor],
+            weight: torch.Tensor, logits: Optional[torch.Tensor] = None,
+            ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """logits [B, vocab] fp32 = RMSNorm(x_rows, final_norm) weight^T (weight: [vocab, H])."""
+    B, vocab = x_rows.shape[0], weight.shape[0]
+    if logits is None:
+        logits = torch.empty((B, vocab), dtype=torch.float32, device=x_rows.device)
+    if ws is None:
+        n = int(lib().q3vl_lm_head_workspace_bytes(ctypes.byref(cfg), B))
+        if n == 0:
+            _check(_abi.EINVAL)
+        ws = torch.empty(n, dtype=torch.uint8, device=x_rows.device)
+    _check(lib().q3vl_lm_head(ctypes.byref(cfg), _ptr(x_rows), B, _ptr(final_norm), _ptr(weight),
+                             vocab, _ptr(logits), _ptr(ws), ws.numel(), _stream(stream)))
+    return logits
+
+
+# ---------------------------------------------------------------------------
 # Step-level calls
 # ---------------------------------------------------------------------------
 def rope_table(cfg: Config, pos: torch.Tensor, stream=None) -> torch.Tensor:

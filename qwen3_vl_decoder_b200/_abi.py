@@ -85,6 +85,9 @@ SIGNATURES = {
     "q3vl_stack_decode": (ctypes.c_int, [_CFG, _I32, ctypes.POINTER(Layer), _P, _P, _I32, _P,
                                          ctypes.POINTER(KvCache), _P, _P, _P, _SZ, _P]),
     "q3vl_decode_advance": (ctypes.c_int, [_I32, _P, _P, _P]),
+    "q3vl_embed": (ctypes.c_int, [_CFG, _P, _I64, _P, _I64, _P, _P, _I32, _P, _P, _SZ, _P]),
+    "q3vl_lm_head_workspace_bytes": (_SZ, [_CFG, _I32]),
+    "q3vl_lm_head": (ctypes.c_int, [_CFG, _P, _I32, _P, _P, _I64, _P, _P, _SZ, _P]),
     "q3vl_device_status": (ctypes.c_int, [_P, ctypes.POINTER(_I32), ctypes.POINTER(_I32)]),
     "q3vl_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_uint32, _P]),
     "q3vl_set_stage_events": (ctypes.c_int, [ctypes.POINTER(_P), _I32]),

@@ -867,6 +867,65 @@ int q3vl_stack_decode(const q3vl_config* cfg, int32_t n_layers, const q3vl_layer
   return Q3VL_OK;
 }
 
+int q3vl_embed(const q3vl_config* cfg, const void* table, int64_t vocab, const int32_t* tokens,
+               int64_t S, const void* soft, const int32_t* soft_rows, int32_t n_soft, void* x,
+               void* ws, size_t ws_bytes, q3vl_stream stream) {
+  Q3VL_TRY(check_cfg(cfg));
+  Q3VL_TRY(check_seq(S));
+  if (vocab < 1) return set_error(Q3VL_EINVAL, "vocab must be >= 1");
+  Q3VL_TRY(check_ptr(table, "table"));
+  Q3VL_TRY(check_ptr(tokens, "tokens", false));
+  Q3VL_TRY(check_ptr(x, "x"));
+  if (n_soft < 0) return set_error(Q3VL_EINVAL, "n_soft must be >= 0");
+  const cudaStream_t st = ST(stream);
+  int32_t* map = nullptr;
+  if (n_soft > 0) {
+    Q3VL_TRY(check_ptr(soft, "soft"));
+    Q3VL_TRY(check_ptr(soft_rows, "soft_rows", false));
+    if (n_soft > S) return set_error(Q3VL_ERANGE, "more soft-token rows than tokens");
+    if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255) != 0 ||
+        ws_bytes < size_t(S) * sizeof(int32_t))
+      return set_error(Q3VL_EWORKSPACE, "embed with soft tokens needs >= 4*S bytes of workspace");
+    map = static_cast<int32_t*>(ws);
+    Q3VL_CUDA(launch_deepstack_map(soft_rows, n_soft, S, map, st), "soft-token row map");
+  }
+  return cuda_check(launch_embed(*cfg, table, vocab, tokens, S, soft, map, x, st), "embed");
+}
+
+size_t q3vl_lm_head_workspace_bytes(const q3vl_config* cfg, int32_t B) {
+  if (check_cfg(cfg) != Q3VL_OK || cfg->dtype != Q3VL_DTYPE_BF16 || check_batch(B) != Q3VL_OK)
+    return 0;
+  return align256(size_t(B) * cfg->hidden * 2);
+}
+
+int q3vl_lm_head(const q3vl_config* cfg, const void* x, int32_t B, const void* final_norm,
+                 const void* weight, int64_t vocab, float* logits, void* ws, size_t ws_bytes,
+                 q3vl_stream stream) {
+  Q3VL_TRY(check_cfg(cfg));
+  if (cfg->dtype != Q3VL_DTYPE_BF16)
+    return set_error(Q3VL_EUNSUPPORTED, "the LM head is bf16 only");
+  Q3VL_TRY(check_batch(B));
+  if (vocab < 1 || vocab > (int64_t(1) << 30)) return set_error(Q3VL_EINVAL, "vocab out of range");
+  Q3VL_TRY(check_ptr(x, "x"));
+  Q3VL_TRY(check_ptr(weight, "weight"));
+  Q3VL_TRY(check_ptr(logits, "logits", false));
+  if (final_norm != nullptr) Q3VL_TRY(check_ptr(final_norm, "final_norm"));
+  const size_t need = align256(size_t(B) * cfg->hidden * 2);
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255) != 0 || ws_bytes < need)
+    return set_error(Q3VL_EWORKSPACE, "lm head workspace too small: need " +
+                                          std::to_string(need) + " bytes");
+  const cudaStream_t st = ST(stream);
+  // the rows, normalised in the workspace (x itself is left as it is)
+  Q3VL_CUDA(cudaMemcpyAsync(ws, x, size_t(B) * cfg->hidden * 2, cudaMemcpyDeviceToDevice, st),
+            "lm head rows");
+  if (final_norm != nullptr)
+    Q3VL_CUDA(launch_final_norm(*cfg, ws, B, final_norm, st), "lm head final norm");
+  DecGemmArgs a{};
+  a.W = weight; a.rows = vocab; a.K = cfg->hidden; a.X = ws; a.B = B;
+  a.N = vocab; a.out = logits;
+  return cuda_check(launch_decode_gemm(Epi::kPlain, a, st), "lm head");
+}
+
 int q3vl_decode_advance(int32_t B, int32_t* pos, int32_t* len, q3vl_stream stream) {
   Q3VL_TRY(check_batch(B));
   Q3VL_TRY(check_ptr(pos, "pos", false));

@@ -49,6 +49,7 @@ struct DecGemmParams {
   // epilogue
   int64_t N;             // output columns (kQkv: q columns nh*128; kSwiGLU: I)
   __nv_bfloat16* out;    // [B][N]
+  float* out_f32;        // [B][N] (kPlain)
   const __nv_bfloat16* resid;  // [B][N] (kResidual)
   float* rowsq_out;      // [B][N/128] (kResidual) or null
   const float* rowsq_in; // [B][rowsq_n] (kQkv, kSwiGLU) or null
@@ -150,6 +151,13 @@ __device__ __forceinline__ void dec_epilogue_token(const DecGemmParams& p, int t
       ss = warp_sum(ss);
       if (lane == 0) p.rowsq_out[int64_t(j) * (p.N / 128) + tile] = ss;
     }
+  } else if constexpr (EPI == static_cast<int>(Epi::kPlain)) {
+    // fp32 rows of N outputs (the last tile may run past N)
+    float* o = p.out_f32 + int64_t(j) * p.N + int64_t(tile) * 128;
+    const int64_t left = p.N - int64_t(tile) * 128;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (lane + 32 * i < left) o[lane + 32 * i] = v[0][i];
   } else {  // kSwiGLU: block 0 = gate rows, block 1 = the matching up rows
     const float s = dec_row_scale(p, j);
     __nv_bfloat16* o = p.out + int64_t(j) * p.N + int64_t(tile) * 128;
@@ -671,7 +679,7 @@ DecSched dec_gemm_sched(int64_t rows, int64_t K, int B, int R) {
   DecSched s{};
   s.R = R;
   s.NB = (B + 15) / 16 * 16;
-  s.tiles = static_cast<int>(rows / (128 * R));
+  s.tiles = static_cast<int>((rows + 128 * R - 1) / (128 * R));  // TMA zero-fills past `rows`
   s.n_k = static_cast<int>((K + kBK - 1) / kBK);
   const size_t stage = size_t(16384) * R + size_t(s.NB) * 128;
   // up to ~110 KB of stages, so that two CTAs share an SM
@@ -770,6 +778,7 @@ cudaError_t launch_dec_epi(const DecGemmArgs& a, int R, cudaStream_t st) {
   p.n_k = s.n_k; p.splits = s.splits; p.stages = s.stages;
   p.err = device_error_ptr();
   p.N = a.N; p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.out_f32 = static_cast<float*>(a.out);
   p.resid = static_cast<const __nv_bfloat16*>(a.resid);
   p.rowsq_out = a.rowsq_out; p.rowsq_in = a.rowsq_in; p.rowsq_n = a.rowsq_n;
   p.rowsq_width = a.rowsq_width; p.inv = a.inv; p.eps = a.eps;
@@ -808,6 +817,7 @@ cudaError_t launch_decode_gemm(Epi epi, const DecGemmArgs& a, cudaStream_t st) {
     case Epi::kQkv: return launch_dec_epi<static_cast<int>(Epi::kQkv)>(a, 1, st);
     case Epi::kResidual: return launch_dec_epi<static_cast<int>(Epi::kResidual)>(a, 1, st);
     case Epi::kSwiGLU: return launch_dec_epi<static_cast<int>(Epi::kSwiGLU)>(a, 2, st);
+    case Epi::kPlain: return launch_dec_epi<static_cast<int>(Epi::kPlain)>(a, 1, st);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -363,6 +363,45 @@ cudaError_t launch_deepstack_map(const int32_t* rows, int n_img, int64_t S, int3
 }
 
 // ---------------------------------------------------------------------------
+// Token embedding gather with the soft-token splice (hf2q
+// qwen3vl_text/forward.rs, `forward_text_prefill_logits_last` step 1):
+// x[p] = table[tokens[p]], except rows with map[p] = k >= 0, which take
+// soft[k]. One warp per row, 16-byte copies. A token id outside the table
+// records Q3VL_ERANGE and leaves the row zero.
+// ---------------------------------------------------------------------------
+__global__ void embed_kernel(const uint4* __restrict__ table, int64_t vocab,
+                             const int32_t* __restrict__ tokens, int64_t S,
+                             const uint4* __restrict__ soft, const int32_t* __restrict__ map,
+                             int64_t row_vecs, uint4* __restrict__ x, int32_t* err) {
+  const int64_t row = int64_t(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= S) return;
+  const uint4* src = nullptr;
+  const int32_t k = map != nullptr ? map[row] : -1;
+  if (k >= 0) {
+    src = soft + int64_t(k) * row_vecs;
+  } else {
+    const int32_t tok = tokens[row];
+    if (tok >= 0 && tok < vocab) src = table + int64_t(tok) * row_vecs;
+    else if (lane == 0) record_error(err, Q3VL_ERANGE, kWhereEmbed);
+  }
+  uint4* dst = x + row * row_vecs;
+  for (int64_t v = lane; v < row_vecs; v += 32)
+    dst[v] = src != nullptr ? __ldg(src + v) : make_uint4(0, 0, 0, 0);
+}
+
+cudaError_t launch_embed(const q3vl_config& c, const void* table, int64_t vocab,
+                         const int32_t* tokens, int64_t S, const void* soft, const int32_t* map,
+                         void* x, cudaStream_t st) {
+  const int64_t row_vecs = int64_t(c.hidden) * int64_t(elem_bytes(c)) / 16;
+  const int warps = 8;
+  embed_kernel<<<static_cast<unsigned>((S + warps - 1) / warps), warps * 32, 0, st>>>(
+      static_cast<const uint4*>(table), vocab, tokens, S, static_cast<const uint4*>(soft), map,
+      row_vecs, static_cast<uint4*>(x), device_error_ptr());
+  return counted_launch(1);
+}
+
+// ---------------------------------------------------------------------------
 // Weight packing (one-time).
 // ---------------------------------------------------------------------------
 enum PackMode : int { kConcat3 = 0, kInterleaveGU = 1, kCopy = 2 };

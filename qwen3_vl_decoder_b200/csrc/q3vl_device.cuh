@@ -19,7 +19,7 @@ constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s
 enum WhereTag : int32_t {
   kWhereGemmProducer = 101, kWhereGemmMma = 102, kWhereGemmEpilogue = 103, kWhereGemmDrain = 104,
   kWhereAttnProducer = 201, kWhereAttnMma = 202, kWhereAttnSoftmax = 203, kWhereAttnDrain = 204,
-  kWherePositions = 301, kWhereDeepstackMap = 302, kWhereSelftest = 401,
+  kWherePositions = 301, kWhereDeepstackMap = 302, kWhereEmbed = 303, kWhereSelftest = 401,
   kWhereDecodeProducer = 501, kWhereDecodeMma = 502, kWhereDecodeEpilogue = 503,
   kWhereDecodeRange = 504, kWhereDecodeAttn = 505,
 };

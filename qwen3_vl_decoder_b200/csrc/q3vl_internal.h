@@ -76,6 +76,9 @@ cudaError_t launch_deepstack_map(const int32_t* rows, int n_img, int64_t S, int3
                                  cudaStream_t st);
 cudaError_t launch_pack(const q3vl_config& c, const q3vl_raw_weights& raw, void* packed,
                         cudaStream_t st);
+cudaError_t launch_embed(const q3vl_config& c, const void* table, int64_t vocab,
+                         const int32_t* tokens, int64_t S, const void* soft, const int32_t* map,
+                         void* x, cudaStream_t st);
 cudaError_t launch_selftest_timeout(uint32_t timeout_us, cudaStream_t st);
 
 // bf16 tensor-core path (tcgen05 + TMA).
@@ -157,7 +160,7 @@ struct DecGemmArgs {
   const void* X;        // bf16 [B, K] tokens
   int B;
   int64_t N;            // output row stride / columns
-  void* out;
+  void* out;            // bf16, or fp32 for kPlain (the LM head's logits)
   const void* resid;
   float* rowsq_out;
   const float* rowsq_in;

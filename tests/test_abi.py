@@ -177,3 +177,27 @@ def test_decode_argument_checks(lib):
     assert pk(65, 0) == -2
     assert pk(8, 2) == -2
     assert pk(8, -1) == -2
+
+
+def test_embed_and_lm_head_argument_checks(lib):
+    c = _cfg()
+    P = ctypes.c_void_p(256)
+    assert lib.q3vl_lm_head_workspace_bytes(ctypes.byref(c), 3) == 3 * 2560 * 2
+    assert lib.q3vl_lm_head_workspace_bytes(ctypes.byref(c), 0) == 0
+    assert lib.q3vl_lm_head_workspace_bytes(ctypes.byref(_cfg(dtype="fp32")), 1) == 0
+
+    def head(cfg=c, B=1, vocab=1000, ws_bytes=1 << 20):
+        return lib.q3vl_lm_head(ctypes.byref(cfg), P, B, None, P, vocab, P, P, ws_bytes, None)
+    assert head(cfg=_cfg(dtype="fp32")) == -8
+    assert head(B=0) == -1 and head(B=257) == -1
+    assert head(vocab=0) == -1
+    assert head(ws_bytes=100) == -5
+
+    def emb(vocab=10, S=4, n_soft=0, ws=None, ws_bytes=0):
+        return lib.q3vl_embed(ctypes.byref(c), P, vocab, P, S, P if n_soft else None,
+                              P if n_soft else None, n_soft, P, ws, ws_bytes, None)
+    assert emb(vocab=0) == -1
+    assert emb(S=0) == -1
+    assert emb(n_soft=-1) == -1
+    assert emb(n_soft=2) == -5                                   # soft rows need the row map
+    assert emb(n_soft=5, ws=P, ws_bytes=1024) == -2              # more soft rows than tokens
