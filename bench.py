@@ -242,7 +242,8 @@ class E2EPipeline:
 def barrier(world):
     if world > 1:
         torch.distributed.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
 
 
 def max_over_ranks(v, world, dev):
