@@ -360,6 +360,7 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
 // ---------------------------------------------------------------------------
 constexpr int kAttnCH = 128;
 constexpr int kAttnThreads = 256;
+constexpr int kAttnTcMinBatch = 2;  // from this batch on, the tcgen05 attention kernel (measured)
 constexpr int kAttnRows = 130;  // per (b, g, h): o[128], m, l, each over the chunk slots
 
 struct DecAttnParams {
@@ -647,6 +648,374 @@ decode_attn_kernel(DecAttnParams p) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// The same attention with the two contractions on tcgen05, for batches with
+// many work items. The cache rows are the MMA's M operand, so the G <= 8
+// query heads of KV head g only pad N to 16:
+//   S^T [128 rows x 16] = K_chunk [128 x 128] . Q^T        (K-major A and B)
+//   O^T [128 dims x 16] = V_chunk^T [128 x 128] . P^T      (V as an MN-major A)
+// K and V arrive by TMA (128-byte swizzle); thread t owns TMEM lane t (cache
+// row t for the softmax, dimension t for the output). An item issues a few
+// hundred instructions per thread instead of the CUDA-core kernel's ~1.8k,
+// but runs its chain (load, S, softmax, O) serially, so three CTAs share an
+// SM to overlap one another's chains. An item here is a contiguous range of
+// chunks of one (b, g) (the host splits each group into about as many items
+// as fill the CTA slots), merged on the fly in registers (running max, sum
+// and o per head), so only an item's result, not every chunk's, goes through
+// global memory and the ticketed merge of decode_attn_kernel. One sequence
+// (B = 1) has too few groups for that and stays on decode_attn_kernel.
+// ---------------------------------------------------------------------------
+constexpr int kTcThreads = 128;
+constexpr int kAttnBlk = 128 * 64 * 2;     // one [128 rows x 64] bf16 swizzle block (16 KB)
+constexpr int kAttnKV = 4 * kAttnBlk;      // K (2 blocks) + V (2 blocks) of one item
+constexpr int kAttnSmall = 16 * 64 * 2;    // one [16 rows x 64] bf16 swizzle block (2 KB)
+
+struct DecAttnTcParams {
+  const __nv_bfloat16* q;        // [B][nh*128]
+  int64_t cap;
+  int n_seq;
+  const int32_t* seq;
+  const int32_t* len;
+  int B, nkv;
+  int nc_pad;                    // chunk slots per (b, g): ceil(cap / kAttnCH), rounded up to 4
+  float scale_log2;
+  __nv_bfloat16* o;              // [B][nh*128]
+  float* part;                   // [B][nkv][G][kAttnRows][nc_pad]
+  uint32_t* tickets;             // [B][nkv], zero between launches
+  int32_t* err;
+  int nsplit;                    // most splits of one (b, g); nc_pad = nsplit rounded up to 4
+};
+
+// Byte offset of element (row r, column c) in a 128-byte-swizzled tile of
+// 64-column blocks with `block_bytes` per block (rows of 128 bytes).
+__device__ __forceinline__ uint32_t sw128_off(int r, int c, uint32_t block_bytes) {
+  return static_cast<uint32_t>(c >> 6) * block_bytes + static_cast<uint32_t>(r) * 128u +
+         ((static_cast<uint32_t>((c & 63) >> 3) ^ static_cast<uint32_t>(r & 7)) << 4) +
+         static_cast<uint32_t>(c & 7) * 2u;
+}
+
+template <int G>
+__host__ __device__ constexpr size_t attn_tc_smem_bytes(int nc_pad) {
+  return 1024 + size_t(kAttnKV) + 2 * kAttnSmall +               // K/V, Q (P aliases Q)
+         size_t(2) * G * nc_pad * 4 + size_t(4) * 8 * 4 * 2 +   // merge weights; warp partials
+         size_t(3) * G * 4 + (2 * kDecMaxB + 2) * 4 + 64;       // m, l, den; items; barriers
+}
+
+template <int G>
+__global__ void __launch_bounds__(kTcThreads, 3)
+decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, DecAttnTcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint8_t* s_kv = sm;                                      // K0 K1 V0 V1
+  uint8_t* s_q = s_kv + kAttnKV;                           // [16 x 128] as 2 blocks
+  // P^T [16 x 128] reuses Q's tile: Q's reader (the S MMA) completed before P
+  // is written, and P's reader (the O MMA) before the next chunk writes Q
+  uint8_t* s_pt = s_q;
+  float* s_w = reinterpret_cast<float*>(s_q + 2 * kAttnSmall);  // [G][nc_pad]
+  float* s_cl = s_w + G * p.nc_pad;                        // [G][nc_pad]
+  float* s_wm = s_cl + G * p.nc_pad;                       // [4 warps][8]
+  float* s_wl = s_wm + 32;                                 // [4 warps][8]
+  float* s_m = s_wl + 32;
+  float* s_l = s_m + G;
+  float* s_den = s_l + G;
+  int* s_nc = reinterpret_cast<int*>(s_den + G);           // [kDecMaxB] splits per token
+  int* s_pref = s_nc + kDecMaxB;                           // [kDecMaxB + 1]
+  int* s_last = s_pref + kDecMaxB + 1;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(
+      (reinterpret_cast<uintptr_t>(s_last + 1) + 7) & ~uintptr_t(7));
+  uint64_t* kv_full = bars;
+  uint64_t* s_full = bars + 1;
+  uint64_t* o_full = bars + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int nh = G * p.nkv;
+  if (t == 0) {
+    mbar_init(kv_full, 1);
+    mbar_init(s_full, 1);
+    mbar_init(o_full, 1);
+    *s_abort = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 32);   // S^T in columns 0..15, O^T in 16..31
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane_field = static_cast<uint32_t>(warp * 32) << 16;
+
+  griddep_wait();
+  griddep_launch_dependents();
+  // items: (token b, KV head g, split s of b's chunks); each split walks a
+  // contiguous range of 128-row chunks
+  for (int b = t; b < p.B; b += kTcThreads) {
+    const int slot = p.seq[b], L = p.len[b];
+    const bool ok = slot >= 0 && slot < p.n_seq && L >= 0 && static_cast<int64_t>(L) < p.cap;
+    const int nc = ok ? (L + kAttnCH) / kAttnCH : 0;  // chunks of rows 0..L
+    s_nc[b] = nc < p.nsplit ? nc : p.nsplit;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // exclusive prefix of items per token: lane l owns tokens 8l .. 8l+7
+    int loc[8], sum = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int b = 8 * lane + i;
+      loc[i] = sum;
+      sum += b < p.B ? p.nkv * s_nc[b] : 0;
+    }
+    int inc = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    const int excl = inc - sum;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int b = 8 * lane + i;
+      if (b < p.B) s_pref[b] = excl + loc[i];
+    }
+    if (lane == 31) s_pref[p.B] = inc;
+  }
+  __syncthreads();
+  const int total = s_pref[p.B];
+
+  constexpr uint32_t idesc_s = idesc_bf16_f32(128, 16, false, false);
+  constexpr uint32_t idesc_o = idesc_bf16_f32(128, 16, true, false);
+  int k = 0;  // chunks this CTA has processed: the phase of all three barriers
+  for (int it = blockIdx.x; it < total; it += gridDim.x) {
+    // a wait that timed out anywhere in the block ends the walk for all
+    // threads (read after the previous chunk's last barrier, written before it)
+    if (*s_abort) break;
+    int lo = 0, hi = p.B - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_pref[mid] <= it) lo = mid;
+      else hi = mid - 1;
+    }
+    const int b = lo;
+    const int splits = s_nc[b];
+    const int loc = it - s_pref[b];
+    const int g = loc / splits, s = loc % splits;
+    const int L1 = p.len[b] + 1;
+    const int nc = (L1 + kAttnCH - 1) / kAttnCH;
+    const int c0 = static_cast<int>(int64_t(s) * nc / splits);
+    const int c1 = static_cast<int>(int64_t(s + 1) * nc / splits);
+    float m_run[G], l_run[G], o_run[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) { m_run[h] = -INFINITY; l_run[h] = 0.f; o_run[h] = 0.f; }
+
+    for (int c = c0; c < c1; ++c, ++k) {
+      if (*s_abort) break;
+      if (t == 0) {
+        // this chunk's rows; the buffer's readers (the previous chunk's MMAs)
+        // completed before the previous chunk's last barrier
+        const int32_t y = static_cast<int32_t>(int64_t(p.seq[b]) * p.cap + int64_t(c) * kAttnCH);
+        mbar_arrive_expect_tx(kv_full, kAttnKV);
+        tma_load_2d(s_kv, &tmK, kv_full, g * 128, y);
+        tma_load_2d(s_kv + kAttnBlk, &tmK, kv_full, g * 128 + 64, y);
+        tma_load_2d(s_kv + 2 * kAttnBlk, &tmV, kv_full, g * 128, y);
+        tma_load_2d(s_kv + 3 * kAttnBlk, &tmV, kv_full, g * 128 + 64, y);
+      }
+      const int n = min(kAttnCH, L1 - c * kAttnCH);
+      // Q^T operand: rows h < G are the query heads of KV head g, rows G..15 zero
+      for (int ch = t; ch < 16 * 16; ch += kTcThreads) {
+        const int h = ch >> 4, cc = ch & 15;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (h < G)
+          v = *reinterpret_cast<const uint4*>(p.q + int64_t(b) * nh * 128 +
+                                              int64_t(g * G + h) * 128 + cc * 8);
+        *reinterpret_cast<uint4*>(s_q + sw128_off(h, cc * 8, kAttnSmall)) = v;
+      }
+      if (!mbar_wait(kv_full, k & 1, p.err, kWhereDecodeAttn, s_abort)) *s_abort = 1;
+      // rows past the sequence hold whatever the cache had: zero V there (P is
+      // zero there, but 0 * NaN would not be)
+      for (int ch = t; ch < (kAttnCH - n) * 16; ch += kTcThreads) {
+        const int r = n + (ch >> 4), cc = ch & 15;
+        *reinterpret_cast<uint4*>(s_kv + 2 * kAttnBlk + (cc >> 3) * kAttnBlk + r * 128 +
+                                  (cc & 7) * 16) = make_uint4(0, 0, 0, 0);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      if (t == 0 && *s_abort == 0) {
+        tc_fence_after();
+        const uint32_t k0 = smem_u32(s_kv), q0 = smem_u32(s_q);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_bf16_ss(tmem, sdesc_sw128(k0 + (kk >> 2) * kAttnBlk + (kk & 3) * 32, 16, 1024),
+                       sdesc_sw128(q0 + (kk >> 2) * kAttnSmall + (kk & 3) * 32, 16, 1024),
+                       idesc_s, kk > 0 ? 1u : 0u);
+        umma_commit(s_full);
+      }
+      // softmax over the chunk's rows: thread t holds row t's scores of every head
+      float sc[16];
+      {
+        bool w_ok = true;
+        if (lane == 0) w_ok = mbar_wait(s_full, k & 1, p.err, kWhereDecodeAttn, s_abort);
+        w_ok = __shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0) != 0;
+        if (!w_ok) *s_abort = 1;
+        tc_fence_after();
+        uint32_t u[16];
+        tmem_ld16(tmem + lane_field, u);
+        tmem_ld_wait();
+#pragma unroll
+        for (int h = 0; h < 16; ++h)
+          sc[h] = t < n ? __uint_as_float(u[h]) * p.scale_log2 : -INFINITY;
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float wm = warp_max(sc[h]);
+        if (lane == 0) s_wm[warp * 8 + h] = wm;
+      }
+      __syncthreads();
+      float mh[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+        mh[h] = fmaxf(fmaxf(s_wm[h], s_wm[8 + h]), fmaxf(s_wm[16 + h], s_wm[24 + h]));
+      float pr[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        pr[h] = t < n ? ex2_approx(sc[h] - mh[h]) : 0.f;
+        const float ws = warp_sum(pr[h]);
+        if (lane == 0) s_wl[warp * 8 + h] = ws;
+      }
+      // P^T operand: row h, column t (zero for h >= G)
+#pragma unroll
+      for (int h = 0; h < 16; ++h) {
+        const __nv_bfloat16 v = __float2bfloat16_rn(h < G ? pr[h < G ? h : 0] : 0.f);
+        *reinterpret_cast<__nv_bfloat16*>(s_pt + sw128_off(h, t, kAttnSmall)) = v;
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      if (t == 0 && *s_abort == 0) {
+        tc_fence_after();
+        const uint32_t v0 = smem_u32(s_kv + 2 * kAttnBlk), p0 = smem_u32(s_pt);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_bf16_ss(tmem + 16, sdesc_sw128(v0 + kk * 2048, kAttnBlk, 1024),
+                       sdesc_sw128(p0 + (kk >> 2) * kAttnSmall + (kk & 3) * 32, 16, 1024),
+                       idesc_o, kk > 0 ? 1u : 0u);
+        umma_commit(o_full);
+      }
+      float acc[G];
+      {
+        bool w_ok = true;
+        if (lane == 0) w_ok = mbar_wait(o_full, k & 1, p.err, kWhereDecodeAttn, s_abort);
+        w_ok = __shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0) != 0;
+        if (!w_ok) *s_abort = 1;
+        tc_fence_after();
+        uint32_t u[16];
+        tmem_ld16(tmem + lane_field + 16, u);
+        tmem_ld_wait();
+#pragma unroll
+        for (int h = 0; h < G; ++h) acc[h] = __uint_as_float(u[h]);
+      }
+      tc_fence_before();
+      __syncthreads();  // TMEM and the operand tiles are free for the next chunk
+      // merge the chunk into the split's running (m, l, o)
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float lj = s_wl[h] + s_wl[8 + h] + s_wl[16 + h] + s_wl[24 + h];
+        const float M = fmaxf(m_run[h], mh[h]);
+        const float wa = ex2_approx(m_run[h] - M), wb = ex2_approx(mh[h] - M);
+        o_run[h] = o_run[h] * wa + acc[h] * wb;
+        l_run[h] = l_run[h] * wa + lj * wb;
+        m_run[h] = M;
+      }
+    }
+    if (*s_abort) break;
+    __nv_bfloat16* ob = p.o + int64_t(b) * nh * 128 + int64_t(g) * G * 128;
+    float* pb = p.part + (size_t(b) * p.nkv + g) * G * kAttnRows * size_t(p.nc_pad);
+    if (splits == 1) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) ob[h * 128 + t] = __float2bfloat16_rn(o_run[h] / l_run[h]);
+    } else {
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float* ph = pb + size_t(h) * kAttnRows * p.nc_pad;
+        ph[size_t(t) * p.nc_pad + s] = o_run[h];
+        if (t == 0) {
+          ph[size_t(128) * p.nc_pad + s] = m_run[h];
+          ph[size_t(129) * p.nc_pad + s] = l_run[h];
+        }
+      }
+      __threadfence();
+      __syncthreads();
+      if (t == 0) {
+        const uint32_t kt = atomicAdd(p.tickets + b * p.nkv + g, 1u);
+        *s_last = kt == static_cast<uint32_t>(splits - 1);
+        if (*s_last) p.tickets[b * p.nkv + g] = 0;
+      }
+      __syncthreads();
+      if (*s_last) {
+        __threadfence();
+        // split maxima and sums in shared memory, then every thread merges
+        // one dimension of every head with independent 16-byte loads
+        for (int idx = t; idx < G * splits; idx += kTcThreads) {
+          const int h = idx / splits, cc = idx % splits;
+          s_w[h * p.nc_pad + cc] = __ldcg(pb + (size_t(h) * kAttnRows + 128) * p.nc_pad + cc);
+          s_cl[h * p.nc_pad + cc] = __ldcg(pb + (size_t(h) * kAttnRows + 129) * p.nc_pad + cc);
+        }
+        __syncthreads();
+        if (t < G) {
+          float M = -INFINITY;
+          for (int cc = 0; cc < splits; ++cc) M = fmaxf(M, s_w[t * p.nc_pad + cc]);
+          float den = 0.f;
+          for (int cc = 0; cc < splits; ++cc) {
+            const float w = ex2_approx(s_w[t * p.nc_pad + cc] - M);
+            s_w[t * p.nc_pad + cc] = w;
+            den = fmaf(w, s_cl[t * p.nc_pad + cc], den);
+          }
+          s_den[t] = den;
+        }
+        __syncthreads();
+        float num[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) num[h] = 0.f;
+#pragma unroll 4
+        for (int c4 = 0; c4 < splits; c4 += 4) {
+          float4 v[G];
+#pragma unroll
+          for (int h = 0; h < G; ++h)
+            v[h] = __ldcg(reinterpret_cast<const float4*>(
+                pb + (size_t(h) * kAttnRows + t) * p.nc_pad + c4));
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float* wv = s_w + h * p.nc_pad + c4;
+            const float vv[4] = {v[h].x, v[h].y, v[h].z, v[h].w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              if (c4 + u < splits) num[h] = fmaf(wv[u], vv[u], num[h]);
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < G; ++h) ob[h * 128 + t] = __float2bfloat16_rn(num[h] / s_den[h]);
+      }
+    }
+    __syncthreads();  // shared buffers are reused by the next item
+  }
+  // every issued K/V load landed: each chunk waits for its own before going on,
+  // except a chunk cut short by a timeout
+  if (t == 0 && k > 0)
+    mbar_wait(kv_full, (k - 1) & 1, p.err, kWhereDecodeAttn, nullptr);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 32);
+  }
+}
+
 // K/V rows of a prefill (the k and v column ranges of the [S, Ntot] QKV
 // buffer) into rows row0 .. row0+S-1 of a cache, 16 bytes per thread.
 __global__ void kv_store_kernel(const uint4* __restrict__ qkv, int64_t S, int64_t ntot8,
@@ -795,6 +1164,23 @@ cudaError_t launch_dec_epi(const DecGemmArgs& a, int R, cudaStream_t st) {
 }
 
 template <int G>
+cudaError_t launch_attn_tc_g(const CUtensorMap& tmK, const CUtensorMap& tmV,
+                             const DecAttnTcParams& p, int grid, cudaStream_t st) {
+  const size_t smem = attn_tc_smem_bytes<G>(p.nc_pad);
+  static size_t smem_set = 0;  // per instantiation
+  if (smem > smem_set) {
+    const cudaError_t e = cudaFuncSetAttribute(
+        decode_attn_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    smem_set = smem;
+  }
+  const cudaError_t e = launch_pdl(decode_attn_tc_kernel<G>, dim3(grid), dim3(kTcThreads), smem,
+                                   st, 1, tmK, tmV, p);
+  if (e != cudaSuccess) return e;
+  return counted_launch(1);
+}
+
+template <int G>
 cudaError_t launch_attn_g(const DecAttnParams& p, int grid, cudaStream_t st) {
   const size_t smem = attn_smem_bytes<G>(p.nc_pad);
   static size_t smem_set = 0;  // per instantiation
@@ -826,6 +1212,42 @@ cudaError_t launch_decode_attention(const q3vl_config& c, const void* q, const q
                                     const int32_t* seq, const int32_t* len, int B, void* o,
                                     float* part, uint32_t* tickets, int64_t items,
                                     cudaStream_t st) {
+  const int G = c.n_heads / c.n_kv_heads;
+  if (B >= kAttnTcMinBatch) {
+    // many items: the tcgen05 kernel, three CTAs per SM
+    const uint64_t rows = uint64_t(kv.n_seq) * uint64_t(kv.cap), dkv = uint64_t(kv_dim(c));
+    CUtensorMap tmK, tmV;
+    if (!make_tmap_bf16(&tmK, kv.k, rows, dkv, dkv, 64, kAttnCH) ||
+        !make_tmap_bf16(&tmV, kv.v, rows, dkv, dkv, 64, kAttnCH))
+      return cudaErrorInvalidValue;
+    DecAttnTcParams t{};
+    t.q = static_cast<const __nv_bfloat16*>(q);
+    t.cap = kv.cap; t.n_seq = kv.n_seq; t.seq = seq; t.len = len;
+    t.B = B; t.nkv = c.n_kv_heads;
+    // splits per (b, g): about enough items to give each of the three CTA
+    // slots per SM one, never more than the chunks of the longest sequence
+    const int64_t slots = 3 * int64_t(sm_count());
+    const int64_t groups = int64_t(B) * c.n_kv_heads;
+    const int64_t max_nc = (kv.cap + kAttnCH - 1) / kAttnCH;
+    int64_t nsplit = (slots + groups - 1) / groups;
+    if (nsplit > max_nc) nsplit = max_nc;
+    if (nsplit < 1) nsplit = 1;
+    t.nsplit = static_cast<int>(nsplit);
+    t.nc_pad = static_cast<int>((nsplit + 3) / 4 * 4);
+    items = groups * nsplit;
+    t.scale_log2 = static_cast<float>(1.4426950408889634 / 11.313708498984761);
+    t.o = static_cast<__nv_bfloat16*>(o);
+    t.part = part; t.tickets = tickets; t.err = device_error_ptr();
+    const int64_t cap_grid = 3 * int64_t(sm_count());
+    const int grid = static_cast<int>(items < cap_grid ? (items > 0 ? items : 1) : cap_grid);
+    switch (G) {
+      case 1: return launch_attn_tc_g<1>(tmK, tmV, t, grid, st);
+      case 2: return launch_attn_tc_g<2>(tmK, tmV, t, grid, st);
+      case 4: return launch_attn_tc_g<4>(tmK, tmV, t, grid, st);
+      case 8: return launch_attn_tc_g<8>(tmK, tmV, t, grid, st);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   DecAttnParams p{};
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k_cache = static_cast<const __nv_bfloat16*>(kv.k);
