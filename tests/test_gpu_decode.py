@@ -79,7 +79,10 @@ def test_prefill_kv_writes_the_layers_k_and_v(w):
     (syn.Q4B_LAYER, [5, 256, 1000]),               # QKV bias, 4 query heads per KV head
     (syn.Q2B_LAYER, [3 * b + 1 for b in range(40)]),  # batch of 40 (MMA N = 48)
     (syn.Q32B_ENC, [64, 700]),                     # 8 query heads per KV head, H = 5120
-], ids=["2b-b4", "4b-b3", "2b-b40", "32b-b2"])
+    # batches whose items span several 128-row chunks (merged in registers):
+    (syn.Q2B_LAYER, [900 + 3 * b for b in range(16)]),  # 4 splits of ~2 chunks per (b, g)
+    (syn.Q2B_LAYER, [400 + b for b in range(64)]),      # 1 split of 4 chunks per (b, g)
+], ids=["2b-b4", "4b-b3", "2b-b40", "32b-b2", "2b-b16-multichunk", "2b-b64-multichunk"])
 def test_layer_decode_matches_oracle(w, lens):
     m = q3()
     cfg = m.config_of(w)
@@ -103,6 +106,41 @@ def test_layer_decode_matches_oracle(w, lens):
         _check_token(got[b], want[b], host(x_new)[b])
         kg, vg = _cache_rows(kv, b, L + 1, w.n_kv_heads)
         assert rel_l2(kg[L], k_new[b]) <= 1e-2 and rel_l2(vg[L], v_new[b]) <= 1e-2, b
+
+
+@pytest.mark.parametrize("seq_slots", [[2], [3, 0, 5, 1]], ids=["b1-slot2", "b4-scattered"])
+def test_decode_reads_and_writes_the_given_cache_slots(seq_slots):
+    # tokens mapped to scattered slots of a 6-slot cache; the other slots hold
+    # unrelated rows that must not leak into the result or be written
+    m = q3()
+    w = syn.Q2B_LAYER
+    cfg = m.config_of(w)
+    raw, packed = layer_on_device(w)
+    B, n_seq, cap = len(seq_slots), 6, 400
+    kv = m.KvCache(cfg, n_seq=n_seq, cap=cap)
+    g = torch.Generator().manual_seed(21)
+    lens = [150 + 37 * s for s in range(n_seq)]
+    for s in range(n_seq):                        # every slot gets its own prompt
+        xp = torch.randn(lens[s], w.hidden, generator=g).to(torch.bfloat16)
+        m.layer_prefill_kv(cfg, packed, xp.cuda(), _text_pos(0, lens[s]), kv, seq=s)
+    before_k = kv.k.clone()
+    x_new = torch.randn(B, w.hidden, generator=g).to(torch.bfloat16)
+    my_lens = [lens[s] for s in seq_slots]
+    xd = x_new.cuda().clone()
+    pos = torch.tensor([my_lens, my_lens, my_lens], dtype=torch.int32).cuda()
+    m.layer_decode(cfg, packed, xd, pos, kv, torch.tensor(seq_slots, dtype=torch.int32).cuda(),
+                   torch.tensor(my_lens, dtype=torch.int32).cuda())
+    m.check_device()
+    caches = [_cache_rows(kv, s, lens[s], w.n_kv_heads) for s in seq_slots]
+    want, k_new, _ = O.layer_decode(O.Config.of(w), raw, host(x_new), np.array([my_lens] * 3),
+                                    [c[0] for c in caches], [c[1] for c in caches])
+    got = host(xd)
+    for i, s in enumerate(seq_slots):
+        _check_token(got[i], want[i], host(x_new)[i])
+        assert rel_l2(host(kv.k[s, lens[s]]).reshape(-1, HD), k_new[i]) <= 1e-2
+    # only row lens[s] of each used slot changed
+    changed = (kv.k != before_k).any(dim=2).nonzero().tolist()
+    assert sorted(changed) == sorted([s, lens[s]] for s in seq_slots)
 
 
 def test_decode_chain_matches_the_prefill_rows():
