@@ -467,8 +467,7 @@ int run_decode_layer(const q3vl_config& c, const q3vl_layer& w, void* x, int32_t
   // P5 over the cache
   Q3VL_CUDA(launch_decode_attention(c, q, kv, seq, len, B, o,
                                     reinterpret_cast<float*>(ws + L.att_part),
-                                    reinterpret_cast<uint32_t*>(ws + L.att_tickets), L.att_items,
-                                    st),
+                                    reinterpret_cast<uint32_t*>(ws + L.att_tickets), st),
             "decode attention");
   // P6 (+ the row sums of squares of h for P7)
   DecGemmArgs r{};

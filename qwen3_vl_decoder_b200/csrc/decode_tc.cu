@@ -349,322 +349,28 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
 // Attention of one new row per sequence over its cache (cortiq-engine
 // qwen3te.rs `Qwen3Encoder::attention_gemm`, the last row of the causal
 // softmax: every cached row and the new row itself, row maximum subtracted).
-// Work items are (token b, KV head g, chunk c of kAttnCH cache rows); a
-// persistent grid walks them. An item copies its K and V rows into shared
-// memory (cp.async, all in flight at once), forms the scores of the G query
-// heads of KV head g, their maximum m and sum l (base-2 exponent with
-// log2(e)/sqrt(128) folded into q) and the unnormalised o. With one chunk
-// the item writes o / l; otherwise the last item of a (b, g) to finish (a
-// ticket counter) merges the chunks:
-//   o = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c,  M = max_c m_c.
-// ---------------------------------------------------------------------------
-constexpr int kAttnCH = 128;
-constexpr int kAttnThreads = 256;
-constexpr int kAttnTcMinBatch = 2;  // from this batch on, the tcgen05 attention kernel (measured)
-constexpr int kAttnRows = 130;  // per (b, g, h): o[128], m, l, each over the chunk slots
-
-struct DecAttnParams {
-  const __nv_bfloat16* q;        // [B][nh*128]
-  const __nv_bfloat16* k_cache;  // [n_seq][cap][nkv*128]
-  const __nv_bfloat16* v_cache;
-  int64_t cap;
-  int n_seq;
-  const int32_t* seq;
-  const int32_t* len;
-  int B, nkv;
-  int nc_pad;                    // chunk slots per (b, g): ceil(cap / kAttnCH), rounded up to 4
-  float scale_log2;
-  __nv_bfloat16* o;              // [B][nh*128]
-  float* part;                   // [B][nkv][G][kAttnRows][nc_pad]
-  uint32_t* tickets;             // [B][nkv], zero between launches
-};
-
-__device__ __forceinline__ void bf16x8_to_f(const uint4& u, float (&f)[8]) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 t = unpack_bf16x2(w[i]);
-    f[2 * i] = t.x;
-    f[2 * i + 1] = t.y;
-  }
-}
-
-template <int G>
-__host__ __device__ constexpr size_t attn_smem_bytes(int nc_pad) {
-  return size_t(2) * kAttnCH * 128 * 2 + size_t(G) * kAttnCH * 4 + size_t(G) * 128 * 4 +
-         size_t(2) * G * nc_pad * 4 +
-         size_t(3) * G * 4 + (2 * kDecMaxB + 2) * 4;
-}
-
-template <int G>
-__global__ void __launch_bounds__(kAttnThreads, 2)
-decode_attn_kernel(DecAttnParams p) {
-  extern __shared__ __align__(16) uint8_t sm[];
-  __nv_bfloat16* k_s = reinterpret_cast<__nv_bfloat16*>(sm);
-  __nv_bfloat16* v_s = k_s + kAttnCH * 128;
-  float* s_p = reinterpret_cast<float*>(v_s + kAttnCH * 128);   // [G][CH]
-  float* s_red = s_p + G * kAttnCH;                              // [G][128]
-  float* s_w = s_red + G * 128;                                  // [G][nc_pad] maxima, weights
-  float* s_cl = s_w + G * p.nc_pad;                              // [G][nc_pad] chunk sums
-  float* s_m = s_cl + G * p.nc_pad;                              // [G]
-  float* s_l = s_m + G;
-  float* s_den = s_l + G;
-  int* s_nc = reinterpret_cast<int*>(s_den + G);                 // [kDecMaxB]
-  int* s_pref = s_nc + kDecMaxB;                                 // [kDecMaxB + 1]
-  int* s_last = s_pref + kDecMaxB + 1;
-
-  griddep_wait();
-  griddep_launch_dependents();
-  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  const int nh = G * p.nkv;
-  const int64_t dkv = int64_t(p.nkv) * 128;
-
-  for (int b = t; b < p.B; b += kAttnThreads) {
-    const int slot = p.seq[b], L = p.len[b];
-    const bool ok = slot >= 0 && slot < p.n_seq && L >= 0 && static_cast<int64_t>(L) < p.cap;
-    s_nc[b] = ok ? (L + kAttnCH) / kAttnCH : 0;  // chunks of rows 0..L
-  }
-  __syncthreads();
-  if (warp == 0) {
-    // exclusive prefix of items per token: lane l owns tokens 8l .. 8l+7
-    int loc[8], sum = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int b = 8 * lane + i;
-      loc[i] = sum;
-      sum += b < p.B ? p.nkv * s_nc[b] : 0;
-    }
-    int inc = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, inc, o);
-      if (lane >= o) inc += y;
-    }
-    const int excl = inc - sum;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int b = 8 * lane + i;
-      if (b < p.B) s_pref[b] = excl + loc[i];
-    }
-    if (lane == 31) s_pref[p.B] = inc;
-  }
-  __syncthreads();
-  const int total = s_pref[p.B];
-
-  for (int it = blockIdx.x; it < total; it += gridDim.x) {
-    int lo = 0, hi = p.B - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (s_pref[mid] <= it) lo = mid;
-      else hi = mid - 1;
-    }
-    const int b = lo;
-    const int nc = s_nc[b];
-    const int loc = it - s_pref[b];
-    const int g = loc / nc, c = loc % nc;
-    const int j0 = c * kAttnCH;
-    const int n = min(kAttnCH, p.len[b] + 1 - j0);
-    const int64_t row0 = int64_t(p.seq[b]) * p.cap + j0;
-    const __nv_bfloat16* kb = p.k_cache + row0 * dkv + int64_t(g) * 128;
-    const __nv_bfloat16* vb = p.v_cache + row0 * dkv + int64_t(g) * 128;
-
-    // this item's K and V rows -> shared memory, all copies in flight at once
-    for (int idx = t; idx < n * 16; idx += kAttnThreads) {
-      const int r = idx >> 4, piece = idx & 15;
-      cp_async16(k_s + r * 128 + piece * 8, kb + r * dkv + piece * 8);
-      cp_async16(v_s + r * 128 + piece * 8, vb + r * dkv + piece * 8);
-    }
-    cp_async_commit();
-    // Scores: a group of LPK = 2G lanes per cache row, each lane holding D =
-    // 64/G dimensions of every query head (64 values of q per lane).
-    constexpr int LPK = 2 * G, D = 128 / LPK, KPW = 32 / LPK;
-    const int kl = lane % LPK, kr = lane / LPK;
-    float qr[G][D];
-#pragma unroll
-    for (int h = 0; h < G; ++h)
-#pragma unroll
-      for (int e = 0; e < D / 8; ++e) {
-        float f[8];
-        bf16x8_to_f(*reinterpret_cast<const uint4*>(p.q + int64_t(b) * nh * 128 +
-                                                   int64_t(g * G + h) * 128 + kl * D + 8 * e),
-                    f);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) qr[h][8 * e + i] = f[i] * p.scale_log2;
-      }
-    cp_async_wait_all();
-    __syncthreads();
-    // the trip count depends on the warp only (the shuffles need all 32 lanes)
-#pragma unroll 1
-    for (int k0 = KPW * warp; k0 < n; k0 += KPW * (kAttnThreads / 32)) {
-      const int kk = k0 + kr;
-      float d[G];
-#pragma unroll
-      for (int h = 0; h < G; ++h) d[h] = 0.f;
-      if (kk < n) {
-#pragma unroll
-        for (int e = 0; e < D / 8; ++e) {
-          float kf[8];
-          bf16x8_to_f(*reinterpret_cast<const uint4*>(k_s + kk * 128 + kl * D + 8 * e), kf);
-#pragma unroll
-          for (int h = 0; h < G; ++h)
-#pragma unroll
-            for (int i = 0; i < 8; ++i) d[h] = fmaf(qr[h][8 * e + i], kf[i], d[h]);
-        }
-      }
-#pragma unroll
-      for (int h = 0; h < G; ++h)
-#pragma unroll
-        for (int o = LPK / 2; o > 0; o >>= 1) d[h] += __shfl_xor_sync(0xffffffffu, d[h], o);
-      if (kl == 0 && kk < n)
-#pragma unroll
-        for (int h = 0; h < G; ++h) s_p[h * kAttnCH + kk] = d[h];
-    }
-    __syncthreads();
-    for (int h = warp; h < G; h += kAttnThreads / 32) {
-      float m = -INFINITY;
-      for (int kk = lane; kk < n; kk += 32) m = fmaxf(m, s_p[h * kAttnCH + kk]);
-      m = warp_max(m);
-      float l = 0.f;
-      for (int kk = lane; kk < n; kk += 32) {
-        const float e = ex2_approx(s_p[h * kAttnCH + kk] - m);
-        s_p[h * kAttnCH + kk] = e;
-        l += e;
-      }
-      l = warp_sum(l);
-      if (lane == 0) { s_m[h] = m; s_l[h] = l; }
-    }
-    __syncthreads();
-    // o[h][d] = sum_kk p[h][kk] v[kk][d]: thread t takes dimension t % 128 over
-    // rows [64 (t / 128), 64 (t / 128) + 64) of the chunk; the halves meet in
-    // shared memory
-    const int dd = t & 127, half = t >> 7;
-    float acc[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) acc[h] = 0.f;
-    {
-      const int kbeg = half * (kAttnCH / 2);
-      const int kend = min(n, kbeg + kAttnCH / 2);
-      int kk = kbeg;
-#pragma unroll 2
-      for (; kk + 4 <= kend; kk += 4) {
-        float v[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) v[u] = __bfloat162float(v_s[(kk + u) * 128 + dd]);
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float4 pw = *reinterpret_cast<const float4*>(s_p + h * kAttnCH + kk);
-          acc[h] = fmaf(pw.x, v[0], acc[h]);
-          acc[h] = fmaf(pw.y, v[1], acc[h]);
-          acc[h] = fmaf(pw.z, v[2], acc[h]);
-          acc[h] = fmaf(pw.w, v[3], acc[h]);
-        }
-      }
-      for (; kk < kend; ++kk) {
-        const float v = __bfloat162float(v_s[kk * 128 + dd]);
-#pragma unroll
-        for (int h = 0; h < G; ++h) acc[h] = fmaf(s_p[h * kAttnCH + kk], v, acc[h]);
-      }
-    }
-    if (half == 1)
-#pragma unroll
-      for (int h = 0; h < G; ++h) s_red[h * 128 + dd] = acc[h];
-    __syncthreads();
-    if (half == 0)
-#pragma unroll
-      for (int h = 0; h < G; ++h) acc[h] += s_red[h * 128 + dd];
-    __nv_bfloat16* ob = p.o + int64_t(b) * nh * 128 + int64_t(g) * G * 128;
-    float* pb = p.part + (size_t(b) * p.nkv + g) * G * kAttnRows * size_t(p.nc_pad);
-    if (nc == 1) {
-      if (half == 0)
-#pragma unroll
-        for (int h = 0; h < G; ++h) ob[h * 128 + dd] = __float2bfloat16_rn(acc[h] / s_l[h]);
-    } else {
-      if (half == 0)
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          float* ph = pb + size_t(h) * kAttnRows * p.nc_pad;
-          ph[size_t(dd) * p.nc_pad + c] = acc[h];
-          if (dd == 0) {
-            ph[size_t(128) * p.nc_pad + c] = s_m[h];
-            ph[size_t(129) * p.nc_pad + c] = s_l[h];
-          }
-        }
-      __threadfence();
-      __syncthreads();
-      if (t == 0) {
-        const uint32_t k = atomicAdd(p.tickets + b * p.nkv + g, 1u);
-        *s_last = k == static_cast<uint32_t>(nc - 1);
-        if (*s_last) p.tickets[b * p.nkv + g] = 0;
-      }
-      __syncthreads();
-      if (*s_last) {
-        __threadfence();
-        // chunk maxima and weights in shared memory, then every thread merges
-        // one dimension of every head with independent 16-byte loads
-        for (int idx = t; idx < G * nc; idx += kAttnThreads) {
-          const int h = idx / nc, cc = idx % nc;
-          s_w[h * p.nc_pad + cc] = __ldcg(pb + (size_t(h) * kAttnRows + 128) * p.nc_pad + cc);
-          s_cl[h * p.nc_pad + cc] = __ldcg(pb + (size_t(h) * kAttnRows + 129) * p.nc_pad + cc);
-        }
-        __syncthreads();
-        if (t < G) {
-          float M = -INFINITY;
-          for (int cc = 0; cc < nc; ++cc) M = fmaxf(M, s_w[t * p.nc_pad + cc]);
-          float den = 0.f;
-          for (int cc = 0; cc < nc; ++cc) {
-            const float w = ex2_approx(s_w[t * p.nc_pad + cc] - M);
-            s_w[t * p.nc_pad + cc] = w;
-            den = fmaf(w, s_cl[t * p.nc_pad + cc], den);
-          }
-          s_den[t] = den;
-        }
-        __syncthreads();
-        if (half == 0) {
-        float num[G];
-#pragma unroll
-        for (int h = 0; h < G; ++h) num[h] = 0.f;
-#pragma unroll 4
-        for (int c4 = 0; c4 < nc; c4 += 4) {
-          float4 v[G];
-#pragma unroll
-          for (int h = 0; h < G; ++h)
-            v[h] = __ldcg(reinterpret_cast<const float4*>(
-                pb + (size_t(h) * kAttnRows + dd) * p.nc_pad + c4));
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float* wv = s_w + h * p.nc_pad + c4;
-            const float vv[4] = {v[h].x, v[h].y, v[h].z, v[h].w};
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-              if (c4 + u < nc) num[h] = fmaf(wv[u], vv[u], num[h]);
-          }
-        }
-#pragma unroll
-        for (int h = 0; h < G; ++h) ob[h * 128 + dd] = __float2bfloat16_rn(num[h] / s_den[h]);
-        }
-      }
-    }
-    __syncthreads();  // shared buffers are reused by the next item
-  }
-}
-
-// ---------------------------------------------------------------------------
-// The same attention with the two contractions on tcgen05, for batches with
-// many work items. The cache rows are the MMA's M operand, so the G <= 8
-// query heads of KV head g only pad N to 16:
+//
+// The two contractions run on tcgen05 with the cache rows as the MMA's M
+// operand, so the G <= 8 query heads of KV head g only pad N to 16:
 //   S^T [128 rows x 16] = K_chunk [128 x 128] . Q^T        (K-major A and B)
 //   O^T [128 dims x 16] = V_chunk^T [128 x 128] . P^T      (V as an MN-major A)
 // K and V arrive by TMA (128-byte swizzle); thread t owns TMEM lane t (cache
 // row t for the softmax, dimension t for the output). An item issues a few
-// hundred instructions per thread instead of the CUDA-core kernel's ~1.8k,
-// but runs its chain (load, S, softmax, O) serially, so three CTAs share an
-// SM to overlap one another's chains. An item here is a contiguous range of
-// chunks of one (b, g) (the host splits each group into about as many items
-// as fill the CTA slots), merged on the fly in registers (running max, sum
-// and o per head), so only an item's result, not every chunk's, goes through
-// global memory and the ticketed merge of decode_attn_kernel. One sequence
-// (B = 1) has too few groups for that and stays on decode_attn_kernel.
+// hundred instructions per thread (a CUDA-core version took ~1.8k), but runs
+// its chain (load, S, softmax, O) serially, so three CTAs share an SM to
+// overlap one another's chains.
+//
+// A work item is a contiguous range of 128-row chunks of one (token b, KV
+// head g); the host splits each group into about as many items as fill the
+// CTA slots (one per SM when there are fewer groups than SMs). The chunks of
+// an item merge on the fly in registers (running max m, sum l and o per head,
+// base-2 exponents with log2(e)/sqrt(128) applied to S in fp32). A group with
+// one item writes o / l; otherwise the last item of the group to finish (a
+// ticket counter) merges the items:
+//   o = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s,  M = max_s m_s.
 // ---------------------------------------------------------------------------
+constexpr int kAttnCH = 128;    // cache rows per chunk (the MMA's M)
+constexpr int kAttnRows = 130;  // per (b, g, h): o[128], m, l, each over the split slots
 constexpr int kTcThreads = 128;
 constexpr int kAttnBlk = 128 * 64 * 2;     // one [128 rows x 64] bf16 swizzle block (16 KB)
 constexpr int kAttnKV = 4 * kAttnBlk;      // K (2 blocks) + V (2 blocks) of one item
@@ -1091,8 +797,8 @@ DecLayout dec_layout(const q3vl_config& c, int B, int64_t cap) {
   L.h = take(size_t(B) * H * 2);
   L.act = take(size_t(B) * I * 2);
   const int G = c.n_heads / c.n_kv_heads;
+  // partial slots per (b, g): at most one per 128-row chunk of a slot
   const int64_t nc_pad = ((cap + kAttnCH - 1) / kAttnCH + 3) / 4 * 4;
-  L.att_items = int64_t(B) * c.n_kv_heads * ((cap + kAttnCH - 1) / kAttnCH);
   L.att_part = take(size_t(B) * c.n_kv_heads * G * kAttnRows * nc_pad * sizeof(float));
   // the ticket region comes last; each decode call clears it once
   L.att_tickets = take(size_t(B) * c.n_kv_heads * sizeof(uint32_t));
@@ -1180,22 +886,6 @@ cudaError_t launch_attn_tc_g(const CUtensorMap& tmK, const CUtensorMap& tmV,
   return counted_launch(1);
 }
 
-template <int G>
-cudaError_t launch_attn_g(const DecAttnParams& p, int grid, cudaStream_t st) {
-  const size_t smem = attn_smem_bytes<G>(p.nc_pad);
-  static size_t smem_set = 0;  // per instantiation
-  if (smem > smem_set) {
-    const cudaError_t e = cudaFuncSetAttribute(
-        decode_attn_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-    if (e != cudaSuccess) return e;
-    smem_set = smem;
-  }
-  const cudaError_t e =
-      launch_pdl(decode_attn_kernel<G>, dim3(grid), dim3(kAttnThreads), smem, st, 1, p);
-  if (e != cudaSuccess) return e;
-  return counted_launch(1);
-}
-
 }  // namespace
 
 cudaError_t launch_decode_gemm(Epi epi, const DecGemmArgs& a, cudaStream_t st) {
@@ -1210,61 +900,40 @@ cudaError_t launch_decode_gemm(Epi epi, const DecGemmArgs& a, cudaStream_t st) {
 
 cudaError_t launch_decode_attention(const q3vl_config& c, const void* q, const q3vl_kv_cache& kv,
                                     const int32_t* seq, const int32_t* len, int B, void* o,
-                                    float* part, uint32_t* tickets, int64_t items,
-                                    cudaStream_t st) {
+                                    float* part, uint32_t* tickets, cudaStream_t st) {
   const int G = c.n_heads / c.n_kv_heads;
-  if (B >= kAttnTcMinBatch) {
-    // many items: the tcgen05 kernel, three CTAs per SM
-    const uint64_t rows = uint64_t(kv.n_seq) * uint64_t(kv.cap), dkv = uint64_t(kv_dim(c));
-    CUtensorMap tmK, tmV;
-    if (!make_tmap_bf16(&tmK, kv.k, rows, dkv, dkv, 64, kAttnCH) ||
-        !make_tmap_bf16(&tmV, kv.v, rows, dkv, dkv, 64, kAttnCH))
-      return cudaErrorInvalidValue;
-    DecAttnTcParams t{};
-    t.q = static_cast<const __nv_bfloat16*>(q);
-    t.cap = kv.cap; t.n_seq = kv.n_seq; t.seq = seq; t.len = len;
-    t.B = B; t.nkv = c.n_kv_heads;
-    // splits per (b, g): about enough items to give each of the three CTA
-    // slots per SM one, never more than the chunks of the longest sequence
-    const int64_t slots = 3 * int64_t(sm_count());
-    const int64_t groups = int64_t(B) * c.n_kv_heads;
-    const int64_t max_nc = (kv.cap + kAttnCH - 1) / kAttnCH;
-    int64_t nsplit = (slots + groups - 1) / groups;
-    if (nsplit > max_nc) nsplit = max_nc;
-    if (nsplit < 1) nsplit = 1;
-    t.nsplit = static_cast<int>(nsplit);
-    t.nc_pad = static_cast<int>((nsplit + 3) / 4 * 4);
-    items = groups * nsplit;
-    t.scale_log2 = static_cast<float>(1.4426950408889634 / 11.313708498984761);
-    t.o = static_cast<__nv_bfloat16*>(o);
-    t.part = part; t.tickets = tickets; t.err = device_error_ptr();
-    const int64_t cap_grid = 3 * int64_t(sm_count());
-    const int grid = static_cast<int>(items < cap_grid ? (items > 0 ? items : 1) : cap_grid);
-    switch (G) {
-      case 1: return launch_attn_tc_g<1>(tmK, tmV, t, grid, st);
-      case 2: return launch_attn_tc_g<2>(tmK, tmV, t, grid, st);
-      case 4: return launch_attn_tc_g<4>(tmK, tmV, t, grid, st);
-      case 8: return launch_attn_tc_g<8>(tmK, tmV, t, grid, st);
-      default: return cudaErrorInvalidValue;
-    }
-  }
-  DecAttnParams p{};
-  p.q = static_cast<const __nv_bfloat16*>(q);
-  p.k_cache = static_cast<const __nv_bfloat16*>(kv.k);
-  p.v_cache = static_cast<const __nv_bfloat16*>(kv.v);
-  p.cap = kv.cap; p.n_seq = kv.n_seq; p.seq = seq; p.len = len;
-  p.B = B; p.nkv = c.n_kv_heads;
-  p.nc_pad = static_cast<int>(((kv.cap + kAttnCH - 1) / kAttnCH + 3) / 4 * 4);
-  p.scale_log2 = static_cast<float>(1.4426950408889634 / 11.313708498984761);  // log2(e)/sqrt(128)
-  p.o = static_cast<__nv_bfloat16*>(o);
-  p.part = part; p.tickets = tickets;
-  const int64_t cap_grid = 4 * int64_t(sm_count());
-  const int grid = static_cast<int>(items < cap_grid ? (items > 0 ? items : 1) : cap_grid);
-  switch (c.n_heads / c.n_kv_heads) {
-    case 1: return launch_attn_g<1>(p, grid, st);
-    case 2: return launch_attn_g<2>(p, grid, st);
-    case 4: return launch_attn_g<4>(p, grid, st);
-    case 8: return launch_attn_g<8>(p, grid, st);
+  const uint64_t rows = uint64_t(kv.n_seq) * uint64_t(kv.cap), dkv = uint64_t(kv_dim(c));
+  CUtensorMap tmK, tmV;
+  if (!make_tmap_bf16(&tmK, kv.k, rows, dkv, dkv, 64, kAttnCH) ||
+      !make_tmap_bf16(&tmV, kv.v, rows, dkv, dkv, 64, kAttnCH))
+    return cudaErrorInvalidValue;
+  DecAttnTcParams t{};
+  t.q = static_cast<const __nv_bfloat16*>(q);
+  t.cap = kv.cap; t.n_seq = kv.n_seq; t.seq = seq; t.len = len;
+  t.B = B; t.nkv = c.n_kv_heads;
+  // splits per (b, g): with fewer groups than SMs (small batches) about one
+  // item per SM, each a few chunks long, so that fewer partials reach the
+  // merge (measured faster); otherwise fill the three CTA slots per SM;
+  // never more than the chunks of the longest sequence
+  const int64_t groups = int64_t(B) * c.n_kv_heads;
+  const int64_t slots = (groups < sm_count() ? 1 : 3) * int64_t(sm_count());
+  const int64_t max_nc = (kv.cap + kAttnCH - 1) / kAttnCH;
+  int64_t nsplit = (slots + groups - 1) / groups;
+  if (nsplit > max_nc) nsplit = max_nc;
+  if (nsplit < 1) nsplit = 1;
+  t.nsplit = static_cast<int>(nsplit);
+  t.nc_pad = static_cast<int>((nsplit + 3) / 4 * 4);
+  t.scale_log2 = static_cast<float>(1.4426950408889634 / 11.313708498984761);  // log2(e)/sqrt(128)
+  t.o = static_cast<__nv_bfloat16*>(o);
+  t.part = part; t.tickets = tickets; t.err = device_error_ptr();
+  const int64_t items = groups * nsplit;
+  const int64_t cap_grid = 3 * int64_t(sm_count());
+  const int grid = static_cast<int>(items < cap_grid ? items : cap_grid);
+  switch (G) {
+    case 1: return launch_attn_tc_g<1>(tmK, tmV, t, grid, st);
+    case 2: return launch_attn_tc_g<2>(tmK, tmV, t, grid, st);
+    case 4: return launch_attn_tc_g<4>(tmK, tmV, t, grid, st);
+    case 8: return launch_attn_tc_g<8>(tmK, tmV, t, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -147,9 +147,8 @@ struct DecLayout {
   size_t o = 0;         // bf16 [B][Dq]
   size_t h = 0;         // bf16 [B][H]
   size_t act = 0;       // bf16 [B][I]
-  size_t att_part = 0;  // fp32 [att_items][G][132] attention chunk partials
+  size_t att_part = 0;  // fp32 [B][nkv][G][130][splits] attention split partials
   size_t att_tickets = 0;  // uint32 [B][nkv], zero between launches
-  int64_t att_items = 0;
   size_t total = 0;
 };
 DecLayout dec_layout(const q3vl_config& c, int B, int64_t cap);
@@ -183,8 +182,7 @@ struct DecGemmArgs {
 cudaError_t launch_decode_gemm(Epi epi, const DecGemmArgs& a, cudaStream_t st);
 cudaError_t launch_decode_attention(const q3vl_config& c, const void* q, const q3vl_kv_cache& kv,
                                     const int32_t* seq, const int32_t* len, int B, void* o,
-                                    float* part, uint32_t* tickets, int64_t items,
-                                    cudaStream_t st);
+                                    float* part, uint32_t* tickets, cudaStream_t st);
 cudaError_t launch_kv_store(const q3vl_config& c, const void* qkv, int64_t S,
                             const q3vl_kv_cache& kv, int32_t seq, cudaStream_t st);
 cudaError_t launch_decode_advance(int B, int32_t* pos, int32_t* len, cudaStream_t st);
