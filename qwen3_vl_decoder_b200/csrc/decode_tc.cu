@@ -837,12 +837,15 @@ cudaError_t launch_pdl(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_
 template <int EPI>
 cudaError_t launch_dec_epi(const DecGemmArgs& a, int R, cudaStream_t st) {
   const DecSched s = dec_gemm_sched(a.rows, a.K, a.B, R);
-  static size_t smem_set = 0;  // per instantiation
-  if (s.smem > smem_set) {
+  static size_t smem_set[64] = {0};  // per instantiation and device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  size_t& done = smem_set[dev >= 0 && dev < 64 ? dev : 0];
+  if (s.smem > done) {
     const cudaError_t e = cudaFuncSetAttribute(
         decode_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(s.smem));
     if (e != cudaSuccess) return e;
-    smem_set = s.smem;
+    done = s.smem;
   }
   CUtensorMap tmW, tmX;
   if (!make_tmap_bf16(&tmW, a.W, a.rows, a.K, a.K, kBK, 128 * R) ||
@@ -873,12 +876,15 @@ template <int G>
 cudaError_t launch_attn_tc_g(const CUtensorMap& tmK, const CUtensorMap& tmV,
                              const DecAttnTcParams& p, int grid, cudaStream_t st) {
   const size_t smem = attn_tc_smem_bytes<G>(p.nc_pad);
-  static size_t smem_set = 0;  // per instantiation
-  if (smem > smem_set) {
+  static size_t smem_set[64] = {0};  // per instantiation and device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  size_t& done = smem_set[dev >= 0 && dev < 64 ? dev : 0];
+  if (smem > done) {
     const cudaError_t e = cudaFuncSetAttribute(
         decode_attn_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     if (e != cudaSuccess) return e;
-    smem_set = smem;
+    done = smem;
   }
   const cudaError_t e = launch_pdl(decode_attn_tc_kernel<G>, dim3(grid), dim3(kTcThreads), smem,
                                    st, 1, tmK, tmV, p);
