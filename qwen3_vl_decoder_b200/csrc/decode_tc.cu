@@ -1,7 +1,7 @@
 // One-token-per-sequence decode on sm_100a: the KV cache writes of the
-// prefill, the skinny projections (tcgen05, swap-AB, split-K), the
-// split-sequence attention over the cache, and the step that advances
-// positions and lengths.
+// prefill, the skinny projections (tcgen05, swap-AB, split-K; also the LM
+// head's), the attention over the cache (tcgen05, split over the sequence),
+// and the step that advances positions and lengths.
 //
 // Why a decoded token needs no re-run of the prompt: hf2q
 // qwen3vl_text/forward.rs, module doc "Why no KV cache yet" (the generation
@@ -22,10 +22,10 @@
 // partial tile in its shared memory, and after a cluster barrier the CTAs
 // share out the tokens, each summing the partials of its tokens over DSMEM
 // in split order and running the epilogue of the prefill's step: 1/rms,
-// bias, per-head RMSNorm and MRoPE
-// with the K/V rows written into the cache (QKV); residual add and the row
-// sum of squares for the next norm (o-projection, down); SiLU(g) * u
-// (gate/up). The weights of a projection do not depend on the previous
+// bias, per-head RMSNorm and MRoPE with the K/V rows written into the cache
+// (QKV); residual add and the row sum of squares for the next norm
+// (o-projection, down); SiLU(g) * u (gate/up); plain fp32 rows (the LM
+// head's logits). The weights of a projection do not depend on the previous
 // kernel, so each projection is launched as a programmatic dependent of it
 // and starts streaming its weights before that kernel has finished.
 #include "q3vl_device.cuh"
