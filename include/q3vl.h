@@ -1,6 +1,8 @@
 /*
  * q3vl.h -- C ABI of libq3vl: the full-sequence causal prefill of a
- * Qwen3-VL text decoder layer and layer stack on an NVIDIA B200 (sm_100a).
+ * Qwen3-VL text decoder layer and layer stack on an NVIDIA B200 (sm_100a),
+ * a KV cache written by the prefill with one-token decode against it, and
+ * the steps either side of the layers (embedding gather, LM head).
  *
  * Sources of the operations (web pages, cited by title and item):
  *   [P] inferencelayer 0.2.3 src/vision.rs, `mrope_positions` -- positions
@@ -10,8 +12,10 @@
  *       `Qwen3Encoder::mrope_positions`, `Qwen3Encoder::attention_gemm`,
  *       `Qwen3Encoder::encode_with_images`.
  *   [H] hf2q 0.1.1 src/inference/models/qwen3vl_text/forward.rs -- module
- *       doc (per-layer order, bias before the q/k norm) and the DeepStack
- *       validation of `forward_text_prefill_logits_last`.
+ *       doc (per-layer order, bias before the q/k norm; "Why no KV cache
+ *       yet"), and `forward_text_prefill_logits_last`: its DeepStack
+ *       validation, step 1 (embedding lookup and soft-token splice) and
+ *       step 4 (final norm and LM head).
  *
  * Conventions for every call:
  *   - Pointers marked "device" are CUDA device pointers on the current

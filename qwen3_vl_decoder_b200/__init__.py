@@ -1,4 +1,8 @@
-"""qwen3_vl_decoder_b200: Qwen3-VL text-decoder causal prefill on B200 (sm_100a).
+"""qwen3_vl_decoder_b200: the Qwen3-VL text decoder on B200 (sm_100a).
+
+The full-sequence causal prefill of a layer or a stack, a KV cache written by
+the prefill with one-token decode against it, and the steps either side: the
+token-embedding gather with the soft-token splice, and the final norm + LM head.
 
 A thin torch-facing binding of libq3vl's C ABI (include/q3vl.h). torch only
 provides device memory and the current stream; every step runs in the
