@@ -180,3 +180,27 @@ def test_stack_decode_equals_the_re_run_stack():
     # the prefill half of stack_prefill_kv is the plain stack
     out, _ = O.stack_prefill_kv(cfg, Ws, x[:S0], pos, slabs, img, final_norm=g)
     assert np.array_equal(out, O.stack(cfg, Ws, x[:S0], pos, slabs, img, final_norm=g))
+
+
+def test_decode_gqa_equals_replicated_kv_heads():
+    # a layer with nh = 4 query heads over nkv = 2 KV heads decodes exactly as
+    # the same layer with every KV head repeated nh / nkv times (MHA) over an
+    # equally repeated cache: query head h reads KV head h div (nh / nkv)
+    w, cfg = _tiny()
+    W = _weights(w)
+    rep = cfg.n_heads // cfg.n_kv_heads
+    W_mha = dict(W)
+    for name in ("wk", "wv"):
+        blocks = W[name].reshape(cfg.n_kv_heads, HD, -1)
+        W_mha[name] = np.repeat(blocks, rep, axis=0).reshape(cfg.n_heads * HD, -1)
+    cfg_mha = O.Config(cfg.hidden, cfg.n_heads, cfg.n_heads, cfg.intermediate)
+    rng = np.random.default_rng(9)
+    L = 13
+    kc = rng.standard_normal((L, cfg.n_kv_heads, HD))
+    vc = rng.standard_normal((L, cfg.n_kv_heads, HD))
+    x = rng.standard_normal((1, cfg.hidden))
+    pos = np.full((3, 1), 21)
+    gqa, _, _ = O.layer_decode(cfg, W, x, pos, [kc], [vc])
+    mha, _, _ = O.layer_decode(cfg_mha, W_mha, x, pos, [np.repeat(kc, rep, axis=1)],
+                               [np.repeat(vc, rep, axis=1)])
+    assert np.allclose(gqa, mha, rtol=1e-13, atol=1e-13)
