@@ -59,6 +59,8 @@ def parse():
     ap.add_argument("--workload", default=syn.Q4B_LAYER.name, choices=sorted(syn.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-stacks", action="store_true",
+                    help="skip the 2B 28-layer stack and 32B 50-layer encoder measurements")
     ap.add_argument("--no-decode", action="store_true",
                     help="skip the one-token decode measurement of the 36-layer stack")
     ap.add_argument("--decode-only", action="store_true",
@@ -114,27 +116,75 @@ def traffic_for_current_kernel():
 
 
 class ClockSampler:
-    """nvidia-smi samples during the timed region (SM clock, throttle reasons)."""
+    """SM clock, power and clock-event reasons sampled during the timed region.
+
+    A thread polls NVML (read-only queries) every few milliseconds between
+    __enter__ and __exit__, so even a timed region of a few tens of
+    milliseconds gets samples. Without NVML it falls back to nvidia-smi.
+    """
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4),
+               ("hw_power_brake_slowdown", 0x80))
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
+    def __init__(self, dev, period_s=0.002):
+        self.dev = dev
+        self.period = period_s
+        self.samples = []      # (sm_mhz, sm_max_mhz, reason mask, power W)
+        self.source = None
         self.proc = None
+        self.out = ""
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(
+                uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.dev.index or 0)
+
+    def _poll(self):
+        nv, h = self.nv, self.h
+        smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self.stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1e3
+                self.samples.append((float(sm), float(smax), int(mask), pw))
+            except Exception:
+                break
+            self.stop.wait(self.period)
 
     def __enter__(self):
+        import threading
+        self.stop = threading.Event()
+        self.thread = None
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            self.nv, self.h = self._nvml_handle()
+            self.source = "nvml"
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.source = "nvidia-smi"
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", "-i", str(self.dev.index or 0), f"--query-gpu={self.FIELDS}",
+                     "--format=csv,noheader,nounits", "-lms", "100"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                time.sleep(0.5)   # its first sample comes a moment after start
+            except OSError:
+                self.proc = None
         return self
 
     def __exit__(self, *a):
-        self.out = ""
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=2)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -142,19 +192,27 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
                 self.out, _ = self.proc.communicate()
+            for r in (self.out or "").strip().splitlines():
+                f = r.split(",")
+                if len(f) < 9:
+                    continue
+                try:
+                    mask = sum(bit for (n, bit), v in zip(self.REASONS[:4], f[5:9])
+                               if v.strip() not in ("", "[N/A]") and "Not" not in v)
+                    self.samples.append((float(f[1]), float(f[2]), mask, float(f[3] or 0)))
+                except ValueError:
+                    continue
 
     def summary(self):
-        rows = [r.split(",") for r in (self.out or "").strip().splitlines() if r.count(",") >= 8]
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
-        sm = [float(r[1]) for r in rows]
-        smax = max(float(r[2]) for r in rows)
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if "Not" not in v
-                          and v.strip() not in ("", "[N/A]")})
-        loaded = [s for s in sm if s > 0.5 * smax] or sm
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax, "reasons": reasons,
-                "samples": len(rows)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"],
+                    "source": self.source}
+        sm = [s[0] for s in self.samples]
+        smax = max(s[1] for s in self.samples)
+        reasons = sorted({n for s in self.samples for n, bit in self.REASONS if s[2] & bit})
+        return {"sm_mhz": statistics.median(sm), "sm_min_mhz": min(sm), "sm_max_mhz": smax,
+                "reasons": reasons, "power_w_max": max(s[3] for s in self.samples),
+                "samples": len(self.samples), "source": self.source}
 
 
 def setup(w, dev):
@@ -445,6 +503,99 @@ def decode_leg(dev, steps, warmup, batches=(1, 32), w=None):
     return out
 
 
+def stack_leg(w, dev, steps, warmup, final_norm_reps=50):
+    """Whole-stack prefill of workload w (all its layers, DeepStack slabs and the
+    final norm as the workload has them), weights drawn and packed on the device.
+    Per-pass time from CUDA events around the stack call (x is restored from a
+    copy between passes, outside the events)."""
+    import qwen3_vl_decoder_b200 as q3
+    cfg = q3.config_of(w)
+    layers = []
+    for l in range(w.n_layers):
+        raw = syn.layer_weights(w, l, device=dev)
+        layers.append(q3.pack_layer(cfg, raw))
+        del raw
+    tt = torch.tensor(syn.token_types(w), dtype=torch.uint8, device=dev)
+    g = syn.grids(w)
+    gd = torch.tensor(g, dtype=torch.int32, device=dev).reshape(-1, 3) if g else None
+    pos, _ = q3.mrope_positions(tt, gd)
+    slabs = [s.to(dev) for s in syn.deepstack_slabs(w)]
+    rows = (torch.tensor(syn.image_rows(w), dtype=torch.int32, device=dev) if slabs else None)
+    gain = syn.final_norm(w, dev)
+    x0 = syn.hidden_input(w, dev)
+    x = x0.clone()
+    ws = q3.workspace(cfg, w.seq, dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for k in range(warmup + steps):
+        x.copy_(x0)
+        if k >= warmup:
+            evs[k - warmup][0].record()
+        q3.stack_prefill(cfg, layers, x, pos, gain, slabs, rows, ws)
+        if k >= warmup:
+            evs[k - warmup][1].record()
+    torch.cuda.synchronize()
+    q3.check_device()
+    assert torch.isfinite(x.float()).all(), f"non-finite {w.name} output"
+    t = statistics.mean(a.elapsed_time(b) for a, b in evs) / 1e3
+    g_f, a_f = layer_flops(w)
+    burst, sustained, hbm, src = peaks()
+    tfl = (g_f + a_f) * w.n_layers / t / 1e12
+    out = {"layers": w.n_layers, "seq_len": w.seq, "final_norm": gain is not None,
+           "deepstack_slabs": len(slabs), "ms_per_stack": 1e3 * t, "steps": steps,
+           "value": w.seq / t, "unit": "tokens/s",
+           "layer_tokens_per_s": w.seq * w.n_layers / t,
+           "tflops": tfl, "frac_of_burst": tfl / burst, "frac_of_sustained": tfl / sustained}
+    if gain is not None:
+        # P10 alone on the stack's output: [S, H] read and written once
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(3):
+            q3.final_norm(cfg, x, gain)
+        e0.record()
+        for _ in range(final_norm_reps):
+            q3.final_norm(cfg, x, gain)
+        e1.record()
+        torch.cuda.synchronize()
+        q3.check_device()
+        tn = e0.elapsed_time(e1) / 1e3 / final_norm_reps
+        nb = 4 * w.seq * w.hidden + 2 * w.hidden
+        out["final_norm_pass"] = {"us": 1e6 * tn, "bytes": nb,
+                                  "roofline": {"bound": "hbm", "achieved": nb / tn / 1e9,
+                                               "peak": hbm, "unit": "GB/s",
+                                               "frac": nb / tn / 1e9 / hbm}}
+    del layers, ws, x, x0
+    torch.cuda.empty_cache()
+    return out
+
+
+def kernel_rooflines(w, stage_ms, peak, peak_name, hbm):
+    """Per-kernel algorithmic work over its live stage time."""
+    S, H, I = w.seq, w.hidden, w.intermediate
+    Dq, Dkv = w.q_dim, w.kv_dim
+    flops = {
+        "qkv": 2 * S * H * (Dq + 2 * Dkv),
+        "attention": 4 * w.n_heads * 128 * S * (S + 1) // 2,
+        "o_proj": 2 * S * Dq * H,
+        "gate_up": 4 * S * H * I,
+        "down": 2 * S * I * H,
+    }
+    out = {}
+    for k, f in flops.items():
+        ms = stage_ms[k]
+        a = f / (ms / 1e3) / 1e12
+        out[k] = {"bound": "tensor", "ms": ms, "gflop": f / 1e9, "achieved": a,
+                  "unit": "TFLOP/s", "peak": peak, "frac": a / peak, "peak_source": peak_name}
+    # the table stage (rope table + stream-K flag clear) and P2 (x read once)
+    hb = {"table": S * 64 * 2 * 4 + 3 * S * 4, "rms1": S * H * 2 + S * 4}
+    for k, b in hb.items():
+        ms = stage_ms[k]
+        if ms > 0:
+            a = b / (ms / 1e3) / 1e9
+            out[k] = {"bound": "hbm", "ms": ms, "bytes": b, "achieved": a, "unit": "GB/s",
+                      "peak": hbm, "frac": a / hbm, "peak_source": "measured copy bandwidth"}
+    return out
+
+
 def main():
     args = parse()
     w = syn.WORKLOADS[args.workload]
@@ -484,11 +635,12 @@ def main():
             e.record()
     torch.cuda.synchronize()
     n0 = q3.launch_count()
-    with ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else 0) as clk:
+    with ClockSampler(dev) as clk:
         t_dev = timed(lambda k: device_step(st, evs[k]), args.steps, world, dev)
     launches = q3.launch_count() - n0
     q3.set_stage_events(None)
     q3.check_device()
+    clocks = clk.summary()
     stage_ms = {name: statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1])
                                       for k in range(args.steps))
                 for i, name in enumerate(STAGES)}
@@ -510,8 +662,14 @@ def main():
     t_e2e = timed(e2e_steps, args.steps, world, dev)
     q3.check_device()
     assert torch.isfinite(st["out_host"].float()).all(), "non-finite output"
+    h2d = st["x_host"].numel() * 2 + st["tt_host"].numel() + \
+        (st["g_host"].numel() * 4 if st["g_host"] is not None else 0)
+    d2h = st["out_host"].numel() * 2
+    del st, pipe
+    torch.cuda.empty_cache()
 
-    # a second workload for reference: the 2B-shape layer at S = 1024 (one GPU only)
+    # the other workloads, for reference (one GPU only): the 2B-shape layer, the
+    # 2B 28-layer stack and the 32B-shape 50-layer encoder at both lengths
     also = {}
     if world == 1 and args.workload != syn.Q2B_LAYER.name:
         w2 = syn.Q2B_LAYER
@@ -526,6 +684,14 @@ def main():
                          "steps": n2, "tflops": (g2 + a2) * n2 / t2 / 1e12}
         del st2
         torch.cuda.empty_cache()
+    if world == 1 and not args.no_stacks:
+        also[syn.Q2B_STACK.name] = stack_leg(syn.Q2B_STACK, dev, steps=10, warmup=3)
+        also[syn.Q32B_ENC_1064.name] = stack_leg(syn.Q32B_ENC_1064, dev, steps=5, warmup=2)
+        also[syn.Q32B_ENC.name] = stack_leg(syn.Q32B_ENC, dev, steps=3, warmup=1)
+        also["context"] = ("the pages time one workload of this path: a 1064-token encode through "
+                           "the 32B-shape encoder truncated at layer 50, 29 s (55 s with the "
+                           "dequantize-and-host-GEMM arm) on a 28-core AVX2 host with quantized "
+                           "weights; context only, not a baseline")
 
     decode = None
     if world == 1 and not args.no_decode:
@@ -534,16 +700,20 @@ def main():
                             syn.Q4B_DECODE.with_layers(args.decode_layers))
 
     burst, sustained, hbm, src = peaks()
+    # The burst peak applies to a kernel timed in a short region at full clock;
+    # the sustained peak (the power-capped clock of a seconds-long loop) when
+    # the timed region is long or the sampled SM clock sat well below its max.
+    at_max = clocks.get("sm_mhz") is not None and clocks["sm_mhz"] >= 0.95 * clocks["sm_max_mhz"]
+    if t_dev < 1.0 or at_max:
+        peak, peak_name = burst, (f"{src} bf16 burst (timed region {t_dev:.3f} s, median SM clock "
+                                  f"{clocks.get('sm_mhz')} of {clocks.get('sm_max_mhz')} MHz)")
+    else:
+        peak, peak_name = sustained, (f"{src} bf16 sustained (timed region {t_dev:.1f} s, median "
+                                      f"SM clock {clocks.get('sm_mhz')} MHz below max)")
     gemm_f, attn_f = layer_flops(w)
-    H, I = w.hidden, w.intermediate
-    gu_flops = 4 * S * H * I
-    gu_s = stage_ms["gate_up"] / 1e3
-    achieved = gu_flops / gu_s / 1e12
+    kr = kernel_rooflines(w, stage_ms, peak, peak_name, hbm)
+    gu = kr["gate_up"]
     tc_s = sum(stage_ms[k] for k in ("qkv", "attention", "o_proj", "gate_up", "down")) / 1e3
-    # P2 (the input row statistic) is the one standalone HBM pass of a bf16
-    # layer: P7 is fused into the o-projection / gate-up epilogues.
-    rms_bytes = S * H * 2 + S * 4
-    rms_gbs = rms_bytes / (stage_ms["rms1"] / 1e3) / 1e9
     if rank != 0:
         if world > 1:
             torch.distributed.destroy_process_group()
@@ -553,10 +723,9 @@ def main():
         n, times = cpu_oracle_rate(w, seconds=10.0)
         cpu = {"value": n * len(times) / sum(times), "unit": UNIT, "cores": cpu_cores(),
                "kind": "oracle",
-               "sample": f"first {n} tokens of {w.name}, fp32 NumPy oracle layer, "
-                         f"{len(times)} passes in {sum(times):.1f} s"}
-    h2d = st["x_host"].numel() * 2 + st["tt_host"].numel() + \
-        (st["g_host"].numel() * 4 if st["g_host"] is not None else 0)
+               "sample": f"first {n} tokens of {w.name} (of {w.seq}), fp32 NumPy oracle layer, "
+                         f"{len(times)} passes in {sum(times):.1f} s; attention cost grows with "
+                         f"S, so the rate overstates the oracle at the full length"}
     line = {
         "metric": METRIC, "value": world * S * args.steps / t_dev, "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -567,27 +736,25 @@ def main():
                    "parallelism": f"replicas x{world}",
                    "l2": "working set larger than L2 (no flush)"},
         "roofline": {"bound": "tensor", "kernel": "gate_up GEMM + SiLU*up epilogue",
-                     "achieved": achieved, "peak": sustained, "unit": "TFLOP/s",
-                     "frac": achieved / sustained,
-                     "peak_source": f"{src} bf16 sustained (timed inside the layer step)",
+                     "achieved": gu["achieved"], "peak": peak, "unit": "TFLOP/s",
+                     "frac": gu["frac"], "peak_source": peak_name,
+                     "frac_of_sustained": gu["achieved"] / sustained,
                      "traffic": traffic_for_current_kernel(),
-                     "flops_per_launch": gu_flops},
+                     "flops_per_launch": gu["gflop"] * 1e9, "ms": gu["ms"]},
+        "kernels": kr,
         "tensor_work": {"gemm_gflop": gemm_f / 1e9, "attn_gflop": attn_f / 1e9,
                         "tflops": (gemm_f + attn_f) / tc_s / 1e12,
-                        "frac_of_sustained": (gemm_f + attn_f) / tc_s / 1e12 / sustained,
-                        "frac_of_burst": (gemm_f + attn_f) / tc_s / 1e12 / burst},
-        "hbm_passes": {"rms1_gbs": rms_gbs, "frac": rms_gbs / hbm, "peak_gbs": hbm,
-                       "bytes": rms_bytes,
-                       "note": "P2 input row statistic, timed with its launch gap; P7 fused "
-                               "into the o-projection epilogue (no pass)"},
+                        "frac": (gemm_f + attn_f) / tc_s / 1e12 / peak,
+                        "frac_of_burst": (gemm_f + attn_f) / tc_s / 1e12 / burst,
+                        "frac_of_sustained": (gemm_f + attn_f) / tc_s / 1e12 / sustained},
         "stages_ms": stage_ms,
         "cpu_baseline": cpu,
         "e2e": {"value": world * S * args.steps / t_e2e, "unit": UNIT,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": st["out_host"].numel() * 2},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "also": also,
         "decode": decode,
         "gpu_launches": launches,
-        "clocks": clk.summary(),
+        "clocks": clocks,
         "next_position": nxt,
     }
     print(json.dumps(line), flush=True)

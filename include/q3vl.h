@@ -188,7 +188,10 @@ int q3vl_stack_prefill(const q3vl_config* cfg, int32_t n_layers, const q3vl_laye
  * whose q3vl_workspace_bytes(cfg, S) exceeds 64 MiB is refused with
  * Q3VL_EWORKSPACE (e.g. the 2B shape fits up to S = 1536 on a 148-SM GPU). The first call on
  * a device looks up the array's device address with that device current;
- * make that first call before any stream capture. All calls share the one
+ * make that first call before any stream capture. The address is kept for
+ * the life of the process: do not call this entry point again on a device
+ * after cudaDeviceReset (or any other teardown of its primary context),
+ * which reloads the library's device code at a new address. All calls share the one
  * array: calls that overlap on the GPU (other streams, other host threads)
  * race on it and must be serialised by the caller. Each call writes every
  * scratch region before reading it, so nothing carries over between calls. */

@@ -12,7 +12,11 @@
 // (64 MiB). Every GPU that loads this library keeps that array for the life
 // of the process. Its device address is looked up once per device, on the
 // first call made with that device current (cudaGetSymbolAddress), so make
-// that first call before any stream capture. All calls share the one array:
+// that first call before any stream capture. The looked-up address is kept
+// for the life of the process, so the entry point must not be used on a
+// device after cudaDeviceReset (or another teardown of its primary context):
+// that reloads this module's device code, and the array, at a new address.
+// All calls share the one array:
 // calls that overlap on the GPU (different streams, or different host
 // threads) race on it and must be serialised by the caller. Nothing in the
 // scratch needs to start at zero: each call writes every scratch region it

@@ -17,6 +17,19 @@ def rel_l2(got, want) -> float:
     return float(np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-300))
 
 
+def max_row_rel(got, want) -> float:
+    """Largest relative L2 error of any single row (last axis): a per-row bound
+    that a handful of wrong rows cannot hide behind the whole-tensor norm."""
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    num = np.linalg.norm((got - want).reshape(-1, want.shape[-1]), axis=1)
+    den = np.maximum(np.linalg.norm(want.reshape(-1, want.shape[-1]), axis=1), 1e-300)
+    return float(np.max(num / den))
+
+
+ROW_TOL_BF16 = 3e-2
+
+
 def max_abs(got, want) -> float:
     return float(np.max(np.abs(np.asarray(got, np.float64) - np.asarray(want, np.float64))))
 

@@ -13,7 +13,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_common import host, positions, q3, rel_l2
+from gpu_common import ROW_TOL_BF16, host, max_row_rel, positions, q3, rel_l2
 from oracle import q3vl_oracle as O
 import q3vl_synth as syn
 
@@ -36,6 +36,8 @@ def _check_layer(w, raw, x_in, x_out, pos_ref, rows, slab=None, ds_rows=None):
     e = rel_l2(got, ref[rows])
     assert e <= 1e-2, e
     assert rel_l2(got - xin, ref[rows] - xin) <= 2e-2
+    assert max_row_rel(got, ref[rows]) <= ROW_TOL_BF16
+    assert max_row_rel(got - xin, ref[rows] - xin) <= 2 * ROW_TOL_BF16
 
 
 def test_2b_stack28_deepstack_final_norm():

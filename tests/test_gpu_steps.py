@@ -9,7 +9,7 @@ import dataclasses
 import numpy as np
 import pytest
 
-from gpu_common import host, layer_on_device, positions, q3, rel_l2
+from gpu_common import ROW_TOL_BF16, host, layer_on_device, max_row_rel, positions, q3, rel_l2
 from oracle import q3vl_oracle as O
 import q3vl_synth as syn
 
@@ -37,6 +37,10 @@ def _within_output_rounding(w, got, ref):
 
 def _tol(w):
     return 2e-6 if w.dtype == "fp32" else 1e-2
+
+
+def _row_tol(w):
+    return 1e-5 if w.dtype == "fp32" else ROW_TOL_BF16
 
 
 @pytest.mark.parametrize("w", CASES, ids=lambda w: f"{w.name}-S{w.seq}")
@@ -69,6 +73,9 @@ def test_steps(w):
     Dq, Dkv = w.q_dim, w.kv_dim
     for name, sl in (("q", slice(0, Dq)), ("k", slice(Dq, Dq + Dkv)), ("v", slice(Dq + Dkv, None))):
         assert rel_l2(got[:, sl], ref[:, sl]) < tol, name
+        # per head row: every (token, head) vector
+        gh, rh = got[:, sl].reshape(-1, 128), ref[:, sl].reshape(-1, 128)
+        assert max_row_rel(gh, rh) < _row_tol(w), (name, max_row_rel(gh, rh))
 
     # P5 attention on the GPU's q, k, v
     o = m.attention(cfg, qkv)
@@ -77,6 +84,8 @@ def test_steps(w):
     vg = got[:, Dq + Dkv:].reshape(S, w.n_kv_heads, 128)
     o_ref = O.attention(qg, kg, vg).reshape(S, -1)
     assert rel_l2(host(o), o_ref) < tol
+    oh, orh = host(o).reshape(-1, 128), o_ref.reshape(-1, 128)
+    assert max_row_rel(oh, orh) < _row_tol(w), max_row_rel(oh, orh)
 
     # P6 o-projection + residual: exact inputs, so the only error is the
     # output's own rounding (half an ulp of bf16 = 2^-8 relative) plus fp32
@@ -90,6 +99,7 @@ def test_steps(w):
     act = m.gate_up(cfg, packed, h, inv2)
     a_ref = O.ffn_act(ocfg, raw, host(h))
     assert rel_l2(host(act), a_ref) < tol
+    assert max_row_rel(host(act), a_ref) < _row_tol(w), max_row_rel(host(act), a_ref)
 
     # P9 down + residual
     out = m.down(cfg, packed, act, h)
