@@ -15,7 +15,10 @@ needed between steps.
             token types copied in, x' copied out, every step (uploads and
             downloads on their own streams, overlapping other steps' kernels);
   roofline  the dominant kernel (gate/up GEMM with SiLU*up epilogue), timed
-            live by stage events the library records inside the timed steps;
+            live by stage events the library records inside every 4th timed
+            step (--stage-every); `kernels` has the same for every kernel;
+  also      the 2B-shape layer, the 2B 28-layer stack and the 32B-shape
+            50-layer encoder (S = 1064 and 8192), with the final-norm pass;
   cpu_baseline the CPU oracle (fp32 NumPy) on a bounded sample.
 
 With N > 1 (torchrun) every rank runs an independent replica on its own GPU
@@ -59,6 +62,8 @@ def parse():
     ap.add_argument("--workload", default=syn.Q4B_LAYER.name, choices=sorted(syn.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--stage-every", type=int, default=4,
+                    help="record the per-kernel stage events on every n-th timed step")
     ap.add_argument("--no-stacks", action="store_true",
                     help="skip the 2B 28-layer stack and 32B 50-layer encoder measurements")
     ap.add_argument("--no-decode", action="store_true",
@@ -240,10 +245,13 @@ def setup(w, dev):
 
 
 def device_step(st, events=None):
+    """P0 and one layer call; with `events` the library records the 9 stage
+    boundaries of this call (and none when events is None)."""
     q3 = st["q3"]
     pos, _ = q3.mrope_positions(st["tt"], st["g"], check=False)
-    if events is not None:
+    if events is not None or st.get("events_on"):
         q3.set_stage_events(events)
+        st["events_on"] = events is not None
     q3.layer_prefill(st["cfg"], st["packed"], st["x"], pos, st["slab"], st["rows"], st["ws"])
 
 
@@ -628,21 +636,27 @@ def main():
         device_step(st)
     q3.check_device()
 
-    # device-resident timed region, with stage events inside every step
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(9)] for _ in range(args.steps)]
-    for row in evs:
+    # Device-resident timed region. Every `stage_every`-th step records the
+    # stage-boundary events the per-kernel times come from. An event between
+    # two kernels keeps the second from starting early as a programmatic
+    # dependent of the first, so those steps run their kernels back to back
+    # without overlap (clean per-kernel times); the other steps do not record.
+    every = max(1, args.stage_every)
+    sampled = [k for k in range(args.steps) if k % every == 0]
+    evs = {k: [torch.cuda.Event(enable_timing=True) for _ in range(9)] for k in sampled}
+    for row in evs.values():
         for e in row:
             e.record()
     torch.cuda.synchronize()
     n0 = q3.launch_count()
     with ClockSampler(dev) as clk:
-        t_dev = timed(lambda k: device_step(st, evs[k]), args.steps, world, dev)
+        t_dev = timed(lambda k: device_step(st, evs.get(k)), args.steps, world, dev)
     launches = q3.launch_count() - n0
     q3.set_stage_events(None)
+    st["events_on"] = False
     q3.check_device()
     clocks = clk.summary()
-    stage_ms = {name: statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1])
-                                      for k in range(args.steps))
+    stage_ms = {name: statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in sampled)
                 for i, name in enumerate(STAGES)}
 
     # end-to-end through the public API with host buffers

@@ -222,7 +222,10 @@ int q3vl_rms_rowstat(const q3vl_config* cfg, const void* x, int64_t S, int64_t w
 
 /* P3+P4. qkv[r] = [q | k | v] of token r, [S, Ntot] in cfg dtype:
  * q,k,v = inv_rms[r] * (x W_qkv^T) + b, then each q and k head is
- * RMS-normalised with q_norm / k_norm and rotated by cos_sin. */
+ * RMS-normalised with q_norm / k_norm and rotated by cos_sin ([S][64][2] as
+ * q3vl_rope_table writes it; a bf16 call first copies it, slot-major, into
+ * the workspace, so it must not overlap the workspace's first
+ * S * 512 bytes). */
 int q3vl_qkv_proj(const q3vl_config* cfg, const q3vl_layer* layer, const void* x, int64_t S,
                   const float* inv_rms, const float* cos_sin, void* qkv, void* ws,
                   size_t ws_bytes, q3vl_stream stream);

@@ -72,7 +72,7 @@ Q2B_STACK = Workload("qwen3vl-2b-stack28-s2048", 2048, 16, 8, 6144, 2048, 28, "b
 Q4B_LAYER = Workload("qwen3vl-4b-layer-s4096", 2560, 32, 8, 9728, 4096, 1, "bf16", 3,
                      qkv_bias=True, images=((512, 32, 24),))
 Q32B_ENC = Workload("qwen3vl-32b-encoder50-s8192", 5120, 64, 8, 25600, 8192, 50, "bf16", 4)
-Q32B_ENC_1064 = Q32B_ENC.with_seq(1064)
+Q32B_ENC_1064 = dataclasses.replace(Q32B_ENC, name="qwen3vl-32b-encoder50-s1064", seq=1064)
 
 WORKLOADS = {w.name: w for w in (TINY_FP32, Q2B_LAYER, Q2B_STACK, Q4B_LAYER, Q32B_ENC,
                                   Q32B_ENC_1064)}

@@ -8,7 +8,10 @@ from __future__ import annotations
 import ctypes
 import os
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libq3vl.so")
+_HERE = os.path.dirname(os.path.abspath(__file__))
+# Q3VL_LIBRARY=debug selects the bounds-checked debug build (libq3vl_debug.so)
+LIB_PATH = os.path.join(_HERE, "libq3vl_debug.so" if os.environ.get("Q3VL_LIBRARY") == "debug"
+                        else "libq3vl.so")
 
 OK, EINVAL, ERANGE, EGRID, EDEEPSTACK, EWORKSPACE, ECUDA, ETIMEOUT, EUNSUPPORTED = \
     0, -1, -2, -3, -4, -5, -6, -7, -8
@@ -99,8 +102,9 @@ SIGNATURES = {
 
 def load(path: str = LIB_PATH) -> ctypes.CDLL:
     if not os.path.exists(path):
-        raise ImportError(f"libq3vl.so is not built ({path}); run "
-                          "`python -m qwen3_vl_decoder_b200.build`")
+        raise ImportError(f"{os.path.basename(path)} is not built ({path}); run "
+                          "`python -m qwen3_vl_decoder_b200.build`"
+                          + (" --debug" if path.endswith("_debug.so") else ""))
     lib = ctypes.CDLL(path)
     for name, (res, args) in SIGNATURES.items():
         fn = getattr(lib, name)

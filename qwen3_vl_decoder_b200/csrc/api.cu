@@ -3,8 +3,10 @@
 // on the caller's stream; nothing here synchronises except
 // q3vl_device_status().
 #include <atomic>
+#include <map>
 #include <mutex>
 #include <string>
+#include <tuple>
 
 #include "q3vl_internal.h"
 
@@ -38,16 +40,66 @@ int cuda_check(cudaError_t e, const char* what) {
 }
 
 int sm_count() {
-  static int cache[64] = {0};
+  static std::atomic<int> cache[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) dev = 0;
-  if (cache[dev] == 0) {
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v == 0) {
     int n = 0;
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    cache[dev] = n > 0 ? n : 148;
+    v = n > 0 ? n : 148;
+    cache[dev].store(v, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return v;
+}
+
+cudaError_t smem_attr_at_least(const void* kernel, size_t bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, size_t> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(mu);
+  size_t& d = done[{kernel, dev}];
+  if (d >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(bytes));
+  if (e == cudaSuccess) d = bytes;
+  return e;
+}
+
+cudaError_t max_active_clusters(const void* kernel, int threads, size_t smem, int cluster,
+                                int* out) {
+  static std::mutex mu;
+  static std::map<std::tuple<const void*, int, size_t, int>, int> cache;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(mu);
+  const auto key = std::make_tuple(kernel, dev, smem, cluster);
+  auto it = cache.find(key);
+  if (it != cache.end()) {
+    *out = it->second;
+    return cudaSuccess;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cluster * (sm_count() / cluster));
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = static_cast<unsigned>(cluster);
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  e = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg);
+  if (e != cudaSuccess) return e;
+  cache[key] = n;
+  *out = n;
+  return cudaSuccess;
 }
 
 WsLayout ws_layout(const q3vl_config& c, int64_t S) {
@@ -322,13 +374,14 @@ int run_down(const q3vl_config& c, const q3vl_layer& w, const void* act, const v
 // already written).
 // `x_stats_ready`: the previous layer of a stack left the row statistics of
 // x in the workspace, so P2 is skipped; `leave_x_stats`: this layer's down
-// epilogue leaves them for the next layer (bf16 path only).
+// epilogue leaves them for the next layer (bf16 path only). `inv1_ready`:
+// the layer prologue already wrote P2's inv_rms.
 // `kv` (optional): the K/V rows of this layer are also written into rows
 // 0..S-1 of slot `kv_seq` of that cache.
 int run_layer(const q3vl_config& c, const q3vl_layer& w, void* x, int64_t S, char* ws,
               const WsLayout& L, const void* ds_slab, cudaStream_t st, bool x_stats_ready = false,
               bool leave_x_stats = false, const q3vl_kv_cache* kv = nullptr,
-              int32_t kv_seq = 0) {
+              int32_t kv_seq = 0, bool inv1_ready = false) {
   float* cs = reinterpret_cast<float*>(ws + L.cos_sin);
   float* inv1 = reinterpret_cast<float*>(ws + L.inv1);
   float* inv2 = reinterpret_cast<float*>(ws + L.inv2);
@@ -340,7 +393,8 @@ int run_layer(const q3vl_config& c, const q3vl_layer& w, void* x, int64_t S, cha
   const Sk sk = sk_of(L, ws);
   float* rowsq_x = is_bf16(c) ? reinterpret_cast<float*>(ws + L.rowsq_x) : nullptr;
   const bool use_x_stats = is_bf16(c) && x_stats_ready;
-  if (!use_x_stats) Q3VL_CUDA(launch_rowstat(c, x, S, c.hidden, inv1, st), "input rms");
+  if (!use_x_stats && !inv1_ready)
+    Q3VL_CUDA(launch_rowstat(c, x, S, c.hidden, inv1, st), "input rms");
   stage_event(2, st);
   Q3VL_TRY(run_qkv(c, w, x, S, inv1, cs, qkv, sk, st, use_x_stats ? rowsq_x : nullptr));
   if (kv != nullptr) Q3VL_CUDA(launch_kv_store(c, qkv, S, *kv, kv_seq, st), "kv cache store");
@@ -367,6 +421,21 @@ int run_layer(const q3vl_config& c, const q3vl_layer& w, void* x, int64_t S, cha
                     is_bf16(c) && leave_x_stats ? rowsq_x : nullptr));
   stage_event(8, st);
   return Q3VL_OK;
+}
+
+// The per-call prologue of a layer or stack: the cos/sin table, the input
+// row statistic of x (bf16: in the same launch) and cleared stream-K flags.
+int run_prologue(const q3vl_config& c, const WsLayout& L, char* ws, const int32_t* pos, int64_t S,
+                 const void* x, cudaStream_t st) {
+  float* cs = reinterpret_cast<float*>(ws + L.cos_sin);
+  if (is_bf16(c)) {
+    const Sk sk = sk_of(L, ws);
+    return cuda_check(launch_layer_prologue(c, pos, S, cs, x, reinterpret_cast<float*>(ws + L.inv1),
+                                            sk.flags, sk.slots, st),
+                      "layer prologue");
+  }
+  Q3VL_TRY(clear_sk_flags(sk_of(L, ws), st));
+  return cuda_check(launch_rope_table(c, pos, S, cs, st), "rope table");
 }
 
 int check_ws(const q3vl_config& c, int64_t S, const void* ws, size_t ws_bytes) {
@@ -596,6 +665,17 @@ int q3vl_qkv_proj(const q3vl_config* cfg, const q3vl_layer* layer, const void* x
   Q3VL_TRY(check_ptr(qkv, "qkv"));
   Sk sk;
   Q3VL_TRY(step_sk(*cfg, S, ws, ws_bytes, ST(stream), &sk));
+  if (is_bf16(*cfg)) {
+    // the bf16 epilogue reads the table slot-major: convert into the workspace
+    float* cs_t = reinterpret_cast<float*>(static_cast<char*>(ws) + ws_layout(*cfg, S).cos_sin);
+    const size_t tb = size_t(S) * kHalf * 2 * sizeof(float);
+    const char* a0 = reinterpret_cast<const char*>(cos_sin);
+    const char* b0 = reinterpret_cast<const char*>(cs_t);
+    if (a0 < b0 + tb && b0 < a0 + tb)
+      return set_error(Q3VL_EINVAL, "cos_sin must not overlap the workspace's table region");
+    Q3VL_CUDA(launch_rope_slot_major(cos_sin, S, cs_t, ST(stream)), "cos/sin slot-major");
+    return run_qkv(*cfg, *layer, x, S, inv_rms, cs_t, qkv, sk, ST(stream));
+  }
   return run_qkv(*cfg, *layer, x, S, inv_rms, cos_sin, qkv, sk, ST(stream));
 }
 
@@ -691,14 +771,13 @@ static int layer_prefill_impl(const q3vl_config* cfg, const q3vl_layer* layer, v
   const WsLayout L = ws_layout(*cfg, S);
   char* w = static_cast<char*>(ws);
   stage_event(0, st);
-  Q3VL_TRY(clear_sk_flags(sk_of(L, w), st));
-  Q3VL_CUDA(launch_rope_table(*cfg, pos, S, reinterpret_cast<float*>(w + L.cos_sin), st),
-            "rope table");
+  Q3VL_TRY(run_prologue(*cfg, L, w, pos, S, x, st));
   if (ds_slab != nullptr)
     Q3VL_CUDA(launch_deepstack_map(ds_rows, n_img, S, reinterpret_cast<int32_t*>(w + L.ds_map), st),
               "deepstack map");
   stage_event(1, st);
-  return run_layer(*cfg, *layer, x, S, w, L, ds_slab, st, false, false, kv, kv_seq);
+  return run_layer(*cfg, *layer, x, S, w, L, ds_slab, st, false, false, kv, kv_seq,
+                   is_bf16(*cfg));
 }
 
 // Cache checks of the *_kv prefill calls: bf16, rows 0..S-1 of one slot.
@@ -763,9 +842,7 @@ static int stack_prefill_impl(const q3vl_config* cfg, int32_t n_layers, const q3
   const cudaStream_t st = ST(stream);
   const WsLayout L = ws_layout(*cfg, S);
   char* w = static_cast<char*>(ws);
-  Q3VL_TRY(clear_sk_flags(sk_of(L, w), st));
-  Q3VL_CUDA(launch_rope_table(*cfg, pos, S, reinterpret_cast<float*>(w + L.cos_sin), st),
-            "rope table");
+  Q3VL_TRY(run_prologue(*cfg, L, w, pos, S, x, st));
   if (n_ds > 0)
     Q3VL_CUDA(launch_deepstack_map(ds_rows, n_img, S, reinterpret_cast<int32_t*>(w + L.ds_map), st),
               "deepstack map");
@@ -775,7 +852,7 @@ static int stack_prefill_impl(const q3vl_config* cfg, int32_t n_layers, const q3
     const void* slab = l < n_ds ? ds_slabs[l] : nullptr;
     // P2 of layer l > 0 comes from layer l-1's down epilogue
     const int rc = run_layer(*cfg, layers[l], x, S, w, L, slab, st, l > 0, l + 1 < n_layers,
-                             kv != nullptr ? kv + l : nullptr, kv_seq);
+                             kv != nullptr ? kv + l : nullptr, kv_seq, l == 0 && is_bf16(*cfg));
     if (rc != Q3VL_OK) g_stage_events_on = events;
     if (rc != Q3VL_OK) return set_error(rc, "layer " + std::to_string(l) + ": " + g_last_error);
   }

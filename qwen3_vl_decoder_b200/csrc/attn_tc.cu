@@ -92,10 +92,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // programmatic dependent launch: let the next kernel start its prologue,
+  // and wait for the QKV projection before reading q, k and v
+  griddep_launch_dependents();
   const uint32_t tO = tmem + 256;
 
   if (warp == 0) {
     if (lane == 0) {
+      griddep_wait();
       mbar_arrive_expect_tx(q_full, kTileBytes);
       tma_load_2d(sQ, &tm, q_full, h * 128, qt * kTile);
       tma_load_2d(sQ + kBlockBytes, &tm, q_full, h * 128 + 64, qt * kTile);
@@ -238,6 +242,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
       tc_fence_before();
       mbar_arrive(p_full);
     }
+    griddep_wait();  // before this kernel's global stores
     if (ok) {
       ok = mbar_wait(o_done, (n_kv - 1) & 1, p.err, kWhereAttnSoftmax, abort_flag);
       if (__all_sync(0xffffffffu, ok)) {
@@ -249,7 +254,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
           uint32_t o[32];
           tmem_ld32(tO + lane_field + 32 * c, o);
           tmem_ld_wait();
-          if (qpos < p.S) {
+          if (qpos < p.S && dcheck((h + 1) * 128 <= p.ldo, p.err, kWhereDbgAttnStore)) {
             uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
 #pragma unroll
             for (int t = 0; t < 4; ++t)
@@ -398,9 +403,13 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // programmatic dependent launch: let the next kernel start its prologue,
+  // and wait for the QKV projection before reading q, k and v
+  griddep_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) {
+      griddep_wait();
       mbar_arrive_expect_tx(q_full, 2 * kTileBytes);
       for (int x = 0; x < 2; ++x) {
         tma_load_2d(sQ + x * kTileBytes, &tm, q_full, (h0 + x) * 128, qt * kTile);
@@ -513,7 +522,7 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
       const bool grow = m_new > m + kRescaleLog2;
       const float m_use = grow ? m_new : m;
       const float alpha = grow ? ex2_approx(m - m_new) : 1.0f;
-      // pass 2: P = 2^(s*scale - m) as bf16 into the first 64 columns of S
+      // P = 2^(s*scale - m) as bf16 into the first 64 columns of S
       const float rs = diag ? exp_regs<true>(sr, tS, r, sc, m_use) : exp_regs<false>(sr, tS, r, sc, m_use);
       l = l * alpha + rs;
       m = m_use;
@@ -533,6 +542,7 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
       tc_fence_before();
       mbar_arrive(p_full + x);
     }
+    griddep_wait();  // before this kernel's global stores
     if (ok) {
       ok = mbar_wait(o_final, 0, p.err, kWhereAttnSoftmax, abort_flag);
       if (__all_sync(0xffffffffu, ok)) {
@@ -544,7 +554,7 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
           uint32_t o[32];
           tmem_ld32(tO + 32 * c, o);
           tmem_ld_wait();
-          if (qpos < p.S) {
+          if (qpos < p.S && dcheck(((h0 + x) + 1) * 128 <= p.ldo, p.err, kWhereDbgAttnStore)) {
             uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
 #pragma unroll
             for (int t = 0; t < 4; ++t)
@@ -586,18 +596,18 @@ cudaError_t launch_attention_tc(const q3vl_config& c, const void* qkv, int64_t S
   p.err = device_error_ptr();
   if ((p.nh / p.nkv) % 2 == 0) {
     // two query heads of one KV group per CTA
-    cudaError_t e = cudaFuncSetAttribute(
-        attn2_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmem2));
+    cudaError_t e = smem_attr_at_least(reinterpret_cast<const void*>(attn2_tc_kernel), kSmem2);
     if (e != cudaSuccess) return e;
     const unsigned grid = static_cast<unsigned>(int64_t(p.num_qt) * (p.nh / 2));
-    attn2_tc_kernel<<<grid, kThreads2, kSmem2, st>>>(tm, p);
+    e = launch_pdl_plain(attn2_tc_kernel, dim3(grid), dim3(kThreads2), kSmem2, st, tm, p);
+    if (e != cudaSuccess) return e;
     return counted_launch(1);
   }
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kSmem));
+  cudaError_t e = smem_attr_at_least(reinterpret_cast<const void*>(attn_tc_kernel), kSmem);
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(int64_t(p.num_qt) * p.nh);
-  attn_tc_kernel<<<grid, kThreads, kSmem, st>>>(tm, p);
+  e = launch_pdl_plain(attn_tc_kernel, dim3(grid), dim3(kThreads), kSmem, st, tm, p);
+  if (e != cudaSuccess) return e;
   return counted_launch(1);
 }
 

@@ -119,6 +119,7 @@ __device__ __forceinline__ void dec_epilogue_token(const DecGemmParams& p, int t
       }
     }
     if (is_q) {
+      if (!dcheck(j < p.B && c0 + 128 <= p.N, p.err, kWhereDbgDecodeStore)) return;
       __nv_bfloat16* o = p.out + int64_t(j) * p.N + c0;
 #pragma unroll
       for (int i = 0; i < 4; ++i) o[lane + 32 * i] = __float2bfloat16_rn(v[0][i]);
@@ -129,6 +130,9 @@ __device__ __forceinline__ void dec_epilogue_token(const DecGemmParams& p, int t
         return;
       }
       const int g = is_k ? tile - p.n_heads : tile - p.n_heads - p.n_kv;
+      if (!dcheck(g >= 0 && g < p.n_kv && slot >= 0 && slot < p.n_seq && row >= 0 &&
+                      row < p.cap, p.err, kWhereDbgDecodeStore))
+        return;
       const int64_t dkv = int64_t(p.n_kv) * 128;
       __nv_bfloat16* dst = (is_k ? p.k_cache : p.v_cache) +
                            (int64_t(slot) * p.cap + row) * dkv + int64_t(g) * 128;
@@ -137,6 +141,7 @@ __device__ __forceinline__ void dec_epilogue_token(const DecGemmParams& p, int t
     }
   } else if constexpr (EPI == static_cast<int>(Epi::kResidual)) {
     const int64_t c0 = int64_t(tile) * 128;
+    if (!dcheck(j < p.B && c0 + 128 <= p.N, p.err, kWhereDbgDecodeStore)) return;
     const __nv_bfloat16* r = p.resid + int64_t(j) * p.N + c0;
     __nv_bfloat16* o = p.out + int64_t(j) * p.N + c0;
     float ss = 0.f;
@@ -160,6 +165,7 @@ __device__ __forceinline__ void dec_epilogue_token(const DecGemmParams& p, int t
       if (lane + 32 * i < left) o[lane + 32 * i] = v[0][i];
   } else {  // kSwiGLU: block 0 = gate rows, block 1 = the matching up rows
     const float s = dec_row_scale(p, j);
+    if (!dcheck(j < p.B && (int64_t(tile) + 1) * 128 <= p.N, p.err, kWhereDbgDecodeStore)) return;
     __nv_bfloat16* o = p.out + int64_t(j) * p.N + int64_t(tile) * 128;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -837,15 +843,10 @@ cudaError_t launch_pdl(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_
 template <int EPI>
 cudaError_t launch_dec_epi(const DecGemmArgs& a, int R, cudaStream_t st) {
   const DecSched s = dec_gemm_sched(a.rows, a.K, a.B, R);
-  static size_t smem_set[64] = {0};  // per instantiation and device
-  int dev = 0;
-  cudaGetDevice(&dev);
-  size_t& done = smem_set[dev >= 0 && dev < 64 ? dev : 0];
-  if (s.smem > done) {
-    const cudaError_t e = cudaFuncSetAttribute(
-        decode_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(s.smem));
+  {
+    const cudaError_t e =
+        smem_attr_at_least(reinterpret_cast<const void*>(decode_gemm_kernel<EPI>), s.smem);
     if (e != cudaSuccess) return e;
-    done = s.smem;
   }
   CUtensorMap tmW, tmX;
   if (!make_tmap_bf16(&tmW, a.W, a.rows, a.K, a.K, kBK, 128 * R) ||
@@ -876,15 +877,10 @@ template <int G>
 cudaError_t launch_attn_tc_g(const CUtensorMap& tmK, const CUtensorMap& tmV,
                              const DecAttnTcParams& p, int grid, cudaStream_t st) {
   const size_t smem = attn_tc_smem_bytes<G>(p.nc_pad);
-  static size_t smem_set[64] = {0};  // per instantiation and device
-  int dev = 0;
-  cudaGetDevice(&dev);
-  size_t& done = smem_set[dev >= 0 && dev < 64 ? dev : 0];
-  if (smem > done) {
-    const cudaError_t e = cudaFuncSetAttribute(
-        decode_attn_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  {
+    const cudaError_t e =
+        smem_attr_at_least(reinterpret_cast<const void*>(decode_attn_tc_kernel<G>), smem);
     if (e != cudaSuccess) return e;
-    done = smem;
   }
   const cudaError_t e = launch_pdl(decode_attn_tc_kernel<G>, dim3(grid), dim3(kTcThreads), smem,
                                    st, 1, tmK, tmV, p);

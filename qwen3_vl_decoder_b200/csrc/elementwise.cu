@@ -55,6 +55,8 @@ positions_kernel(const uint8_t* __restrict__ tt, int64_t S, const int32_t* __res
   __shared__ int32_t s_carry;
   __shared__ int32_t s_max[32];
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  griddep_wait();
+  griddep_launch_dependents();
 
   if (tid == 0) {
     info[0] = 0;
@@ -173,7 +175,10 @@ positions_kernel(const uint8_t* __restrict__ tt, int64_t S, const int32_t* __res
 
 cudaError_t launch_positions(const uint8_t* tt, int64_t S, const int32_t* grids, int n_grids,
                              int32_t* pos, int32_t* info, cudaStream_t st) {
-  positions_kernel<<<1, kPosThreads, 0, st>>>(tt, S, grids, n_grids, pos, info);
+  const cudaError_t e =
+      launch_pdl_plain(positions_kernel, dim3(1), dim3(kPosThreads), 0, st, tt, S, grids, n_grids,
+                       pos, info);
+  if (e != cudaSuccess) return e;
   return counted_launch(1);
 }
 
@@ -275,6 +280,90 @@ cudaError_t launch_rowstat(const q3vl_config& c, const void* x, int64_t S, int64
   else
     rowstat_kernel<float><<<blocks, warps * 32, 0, st>>>(static_cast<const float*>(x), S, width,
                                                          static_cast<float>(c.rms_eps), inv);
+  return counted_launch(1);
+}
+
+// ---------------------------------------------------------------------------
+// The cos/sin table in the slot-major layout the bf16 QKV epilogue reads:
+// float4 number t * S + p holds (cos, sin) of slots 2t and 2t + 1 at
+// position p, so the 32 threads of a warp (32 consecutive rows) read 512
+// contiguous bytes per slot pair. From the position-major [S][64][2] table.
+// ---------------------------------------------------------------------------
+__global__ void rope_slot_major_kernel(const float4* __restrict__ cs, int64_t S,
+                                       float4* __restrict__ out) {
+  const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= S * (kHalf / 2)) return;
+  const int64_t t = idx / S, pp = idx % S;
+  out[t * S + pp] = cs[pp * (kHalf / 2) + t];
+}
+
+cudaError_t launch_rope_slot_major(const float* cs, int64_t S, float* out, cudaStream_t st) {
+  const int64_t n = S * (kHalf / 2);
+  rope_slot_major_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
+      reinterpret_cast<const float4*>(cs), S, reinterpret_cast<float4*>(out));
+  return counted_launch(1);
+}
+
+// ---------------------------------------------------------------------------
+// The bf16 layer's prologue in one launch: P1 (the cos/sin table, written
+// slot-major as above) in blocks
+// [0, table_blocks), P2 (the input row statistic, a warp per row) in the
+// blocks after them, and the stream-K flags of the GEMMs set to zero by
+// block 0. Launched as a programmatic dependent: it waits for the previous
+// kernel in the stream (the positions, or the previous layer) before reading
+// pos or x, and lets the QKV GEMM start its prologue early.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+layer_prologue_kernel(const int32_t* __restrict__ pos, int64_t S, double theta, int sec_h,
+                      int sec_w, float2* __restrict__ cs, int table_blocks,
+                      const __nv_bfloat16* __restrict__ x, int64_t width, float eps,
+                      float* __restrict__ inv, int32_t* __restrict__ flags, int n_flags) {
+  griddep_wait();
+  griddep_launch_dependents();
+  if (static_cast<int>(blockIdx.x) < table_blocks) {
+    __shared__ double freq[kHalf];
+    if (threadIdx.x < kHalf) freq[threadIdx.x] = pow(theta, -2.0 * threadIdx.x / kHeadDim);
+    if (blockIdx.x == 0)
+      for (int i = threadIdx.x; i < n_flags; i += blockDim.x) flags[i] = 0;
+    __syncthreads();
+    // slot-major: consecutive threads take consecutive positions of one slot
+    const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= S * kHalf) return;
+    const int i = static_cast<int>(idx / S);
+    const int64_t pp = idx % S;
+    int axis = 0;
+    if (i % 3 == 1 && i < 3 * sec_h) axis = 1;
+    else if (i % 3 == 2 && i < 3 * sec_w) axis = 2;
+    const double ang = static_cast<double>(pos[axis * S + pp]) * freq[i];
+    double sn, c;
+    sincos(ang, &sn, &c);
+    cs[(int64_t(i >> 1) * S + pp) * 2 + (i & 1)] =
+        make_float2(static_cast<float>(c), static_cast<float>(sn));
+    return;
+  }
+  if (x == nullptr) return;
+  const int64_t row = int64_t(blockIdx.x - table_blocks) * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= S) return;
+  const float sq = row_sumsq<__nv_bfloat16>(reinterpret_cast<const uint4*>(x + row * width),
+                                            width * 2 / 16, lane);
+  if (lane == 0) inv[row] = 1.0f / sqrtf(sq / static_cast<float>(width) + eps);
+}
+
+cudaError_t launch_layer_prologue(const q3vl_config& c, const int32_t* pos, int64_t S, float* cs,
+                                  const void* x, float* inv, int32_t* flags, int n_flags,
+                                  cudaStream_t st) {
+  const int th = 256;
+  const int table_blocks = static_cast<int>((S * kHalf + th - 1) / th);
+  const int rows_per_block = th / 32;
+  const int stat_blocks = x != nullptr ? static_cast<int>((S + rows_per_block - 1) / rows_per_block)
+                                       : 0;
+  const cudaError_t e = launch_pdl_plain(
+      layer_prologue_kernel, dim3(table_blocks + stat_blocks), dim3(th), 0, st, pos, S,
+      c.rope_theta, c.mrope_section[1], c.mrope_section[2], reinterpret_cast<float2*>(cs),
+      table_blocks, static_cast<const __nv_bfloat16*>(x), static_cast<int64_t>(c.hidden),
+      static_cast<float>(c.rms_eps), inv, flags, n_flags);
+  if (e != cudaSuccess) return e;
   return counted_launch(1);
 }
 

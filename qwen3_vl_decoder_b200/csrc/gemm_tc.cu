@@ -26,7 +26,8 @@
 // the bias-before-norm order):
 //   kQkv      v = inv_rms[r] * acc + b; q/k heads: per-head RMSNorm with the
 //             q_norm / k_norm gain, then split-half MRoPE from the cos/sin
-//             table; v heads: v only.
+//             table (slot-major, so a warp's loads are contiguous); v heads:
+//             v only.
 //   kResidual out = resid + acc (+ DeepStack slab row ds_map[r]).
 //   kSwiGLU   out = silu(s*g) * (s*u), s = inv_rms[r] (fast exp / divide); B's 256-row block
 //             holds 128 gate rows then the 128 matching up rows.
@@ -69,11 +70,13 @@ struct Params {
   int32_t* err;
   // schedule over pair tiles (see WorkIter)
   int64_t dp_tiles, sk_units;
+  int sk_pairs;   // pairs 0 .. sk_pairs-1 share the stream-K units
   int kb_per_tile;
   int m_fastest;  // tile order: 1 = M index fastest (A stays in L2), 0 = N fastest (B stays)
   // stream-K scratch: one fp32 128 x BN partial tile and one flag per CTA
   float* sk_partials;
   int32_t* sk_flags;
+  int sk_slots;   // CTA slots of partials and flags (checked by debug builds)
   // row statistics between GEMMs (see GemmArgs)
   float* rowsq_out;
   const float* rowsq_in;
@@ -87,8 +90,8 @@ struct Params {
 //   tiles [0, dp_tiles): data parallel; pair c takes tiles c, c + G, ... over
 //     their whole K range;
 //   tiles [dp_tiles, T): stream-K; their U = (T - dp_tiles) * KB k-block
-//     units are cut into G equal contiguous ranges, pair c taking units
-//     [c U / G, (c + 1) U / G).
+//     units are cut into Gs = sk_pairs equal contiguous ranges, pair c < Gs
+//     taking units [c U / Gs, (c + 1) U / Gs).
 // A stream-K tile split across pairs is finished by the pair holding its
 // first k-block, which reaches it last (at the end of its stream-K range).
 // The pairs holding its later k-blocks reach them first (at the start of
@@ -108,8 +111,10 @@ struct WorkIter {
   int64_t u, u1, sk_base;
   int KB;
   __device__ WorkIter(const Params& p, int c, int G)
-      : dp_t(c), dp_tiles(p.dp_tiles), stride(G), u(p.sk_units * c / G),
-        u1(p.sk_units * (c + 1) / G), sk_base(p.dp_tiles), KB(p.kb_per_tile) {}
+      : dp_t(c), dp_tiles(p.dp_tiles), stride(G),
+        u(c < p.sk_pairs ? p.sk_units * c / p.sk_pairs : 0),
+        u1(c < p.sk_pairs ? p.sk_units * (c + 1) / p.sk_pairs : 0), sk_base(p.dp_tiles),
+        KB(p.kb_per_tile) {}
   __device__ bool next(Work& w) {
     if (u < u1) {
       const int64_t t = u / KB;
@@ -219,67 +224,113 @@ __device__ __forceinline__ void add_bf16x32(float* v, const __nv_bfloat16* src) 
   }
 }
 
+// Layout of a stream-K partial tile in its scratch slot: the float4 holding
+// accumulator columns [32 cc + 4 j, 32 cc + 4 j + 4) of row rr is float4
+// number (cc * 8 + j) * BM + rr, so each warp-wide store or load of one
+// (cc, j) covers 32 consecutive float4 (512 contiguous bytes).
+__device__ __forceinline__ size_t part_f4(int cc, int j, int rr) {
+  return (static_cast<size_t>(cc) * 8 + j) * BM + rr;
+}
+
 // Loads accumulator columns [32 cc, 32 cc + 32) of this thread's row from
 // TMEM and adds the fp32 partial rows of n_part contributor slots (slot i at
-// part + i * slot_stride floats).
-template <int BN>
+// part + i * slot_stride floats). The partials are requested kGroup slots at
+// a time, all before any of them is used, so n_part slots cost about
+// n_part / kGroup round trips to L2 instead of n_part.
+template <int BN, int kGroup>
 __device__ __forceinline__ void load_chunk(uint32_t taddr, int cc, int rr, const float* part,
                                            int n_part, size_t slot_stride, float* v) {
-  float4 q0[8];
-  const size_t off = (static_cast<size_t>(cc) * BM + rr) * 32;
-  if (n_part > 0) {
-    const float4* src = reinterpret_cast<const float4*>(part + off);
+  float4 q[kGroup][8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) q0[j] = __ldcg(src + j);
-  }
+  for (int u = 0; u < kGroup; ++u)
+    if (u < n_part) {
+      const float4* src = reinterpret_cast<const float4*>(part + u * slot_stride);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) q[u][j] = __ldcg(src + part_f4(cc, j, rr));
+    }
   uint32_t r[32];
   tmem_ld32(taddr, r);
   tmem_ld_wait();
 #pragma unroll
   for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(r[t]);
-  if (n_part > 0) {
+  for (int i0 = 0; i0 < n_part; i0 += kGroup) {
+    if (i0 > 0) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      v[4 * j] += q0[j].x; v[4 * j + 1] += q0[j].y; v[4 * j + 2] += q0[j].z; v[4 * j + 3] += q0[j].w;
-    }
-  }
-  for (int i = 1; i < n_part; ++i) {
-    const float4* src = reinterpret_cast<const float4*>(part + i * slot_stride + off);
+      for (int u = 0; u < kGroup; ++u)
+        if (i0 + u < n_part) {
+          const float4* src = reinterpret_cast<const float4*>(part + (i0 + u) * slot_stride);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float4 q = __ldcg(src + j);
-      v[4 * j] += q.x; v[4 * j + 1] += q.y; v[4 * j + 2] += q.z; v[4 * j + 3] += q.w;
+          for (int j = 0; j < 8; ++j) q[u][j] = __ldcg(src + part_f4(cc, j, rr));
+        }
     }
+#pragma unroll
+    for (int u = 0; u < kGroup; ++u)
+      if (i0 + u < n_part) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          v[4 * j] += q[u][j].x; v[4 * j + 1] += q[u][j].y;
+          v[4 * j + 2] += q[u][j].z; v[4 * j + 3] += q[u][j].w;
+        }
+      }
   }
 }
 
-// One 128-column head of the QKV epilogue for this thread's row, staged as
-// chunks [cc0, cc0 + 4) of the epilogue tile.
+// 1 / rms of row `row`: from the per-tile sums of squares of the previous
+// GEMM's epilogue (rowsq_in, summed in tile order) or the given row scale.
+// The partial sums are requested eight at a time before any is added, so the
+// sum costs a few L2 round trips, not one per tile.
+__device__ __forceinline__ float row_inv_rms(const Params& p, int64_t row) {
+  if (p.rowsq_in == nullptr) return p.row_scale[row];
+  const float* rs = p.rowsq_in + row * p.rowsq_n;
+  float ss = 0.f;
+  for (int t0 = 0; t0 < p.rowsq_n; t0 += 8) {
+    float q[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) q[u] = t0 + u < p.rowsq_n ? __ldg(rs + t0 + u) : 0.f;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) ss += q[u];
+  }
+  return 1.0f / sqrtf(ss / p.rowsq_width + p.eps);
+}
+
+// One 128-column head of the QKV epilogue for this thread's row (row scale
+// s), staged as chunks [cc0, cc0 + 4) of the epilogue tile. Every global
+// read (bias, norm gain, cos/sin) is issued eight float4 at a time ahead of
+// its use, so a head costs a dozen round trips to L1/L2 rather than a
+// hundred.
 template <int BN>
 __device__ __forceinline__ void qkv_head(uint32_t taddr, int cc0, int rr, const float* part,
                                          int n_part, size_t slot_stride, int64_t row, bool valid,
-                                         int64_t c0, const Params& p, uint8_t* tile) {
+                                         float s, int64_t c0, const Params& p, uint8_t* tile) {
   float v[128];
+  if (n_part == 0) {
+    // all four TMEM loads in flight at once, one wait (the raw fp32 bits land
+    // in v directly)
 #pragma unroll
-  for (int j = 0; j < 4; ++j)
-    load_chunk<BN>(taddr + 32 * j, cc0 + j, rr, part, n_part, slot_stride, v + 32 * j);
+    for (int j = 0; j < 4; ++j)
+      tmem_ld32(taddr + 32 * j, *reinterpret_cast<uint32_t(*)[32]>(v + 32 * j));
+    tmem_ld_wait();
+  } else {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      load_chunk<BN, 1>(taddr + 32 * j, cc0 + j, rr, part, n_part, slot_stride, v + 32 * j);
+  }
   if (valid) {
-    float s;
-    if (p.rowsq_in != nullptr) {
-      float ss = 0.f;
-      for (int t = 0; t < p.rowsq_n; ++t) ss += p.rowsq_in[row * p.rowsq_n + t];
-      s = 1.0f / sqrtf(ss / p.rowsq_width + p.eps);
-    } else {
-      s = p.row_scale[row];
-    }
 #pragma unroll
     for (int t = 0; t < 128; ++t) v[t] *= s;
     if (p.bias != nullptr) {
       const float4* b = reinterpret_cast<const float4*>(p.bias + c0);
 #pragma unroll
-      for (int t = 0; t < 32; ++t) {
-        const float4 bb = __ldg(b + t);
-        v[4 * t] += bb.x; v[4 * t + 1] += bb.y; v[4 * t + 2] += bb.z; v[4 * t + 3] += bb.w;
+      for (int t0 = 0; t0 < 32; t0 += 4) {
+        float4 bb[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) bb[u] = __ldg(b + t0 + u);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int t = t0 + u;
+          v[4 * t] += bb[u].x; v[4 * t + 1] += bb[u].y;
+          v[4 * t + 2] += bb[u].z; v[4 * t + 3] += bb[u].w;
+        }
       }
     }
     const bool is_q = c0 < p.q_cols;
@@ -291,21 +342,33 @@ __device__ __forceinline__ void qkv_head(uint32_t taddr, int cc0, int rr, const 
       const float rn = 1.0f / sqrtf(ss * (1.0f / 128.0f) + p.eps);
       const float4* g = reinterpret_cast<const float4*>(is_q ? p.q_norm : p.k_norm);
 #pragma unroll
-      for (int t = 0; t < 32; ++t) {
-        const float4 gg = __ldg(g + t);
-        v[4 * t] *= rn * gg.x; v[4 * t + 1] *= rn * gg.y;
-        v[4 * t + 2] *= rn * gg.z; v[4 * t + 3] *= rn * gg.w;
-      }
-      const float4* cs = reinterpret_cast<const float4*>(p.cos_sin + row * 64);
+      for (int t0 = 0; t0 < 32; t0 += 4) {
+        float4 gg[4];
 #pragma unroll
-      for (int t = 0; t < 32; ++t) {
-        const float4 q = __ldg(cs + t);  // (cos_i, sin_i, cos_{i+1}, sin_{i+1}), i = 2t
-        const int i = 2 * t;
-        const float a0 = v[i], b0 = v[i + 64], a1 = v[i + 1], b1 = v[i + 65];
-        v[i] = a0 * q.x - b0 * q.y;
-        v[i + 64] = a0 * q.y + b0 * q.x;
-        v[i + 1] = a1 * q.z - b1 * q.w;
-        v[i + 65] = a1 * q.w + b1 * q.z;
+        for (int u = 0; u < 4; ++u) gg[u] = __ldg(g + t0 + u);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int t = t0 + u;
+          v[4 * t] *= rn * gg[u].x; v[4 * t + 1] *= rn * gg[u].y;
+          v[4 * t + 2] *= rn * gg[u].z; v[4 * t + 3] *= rn * gg[u].w;
+        }
+      }
+      // slot-major table: one warp reads 32 consecutive rows' float4 per slot pair
+      const float4* cs = reinterpret_cast<const float4*>(p.cos_sin) + row;
+#pragma unroll
+      for (int t0 = 0; t0 < 32; t0 += 4) {
+        float4 q[4];  // (cos_i, sin_i, cos_{i+1}, sin_{i+1}), i = 2t
+#pragma unroll
+        for (int u = 0; u < 4; ++u) q[u] = __ldg(cs + int64_t(t0 + u) * p.M);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = 2 * (t0 + u);
+          const float a0 = v[i], b0 = v[i + 64], a1 = v[i + 1], b1 = v[i + 65];
+          v[i] = a0 * q[u].x - b0 * q[u].y;
+          v[i + 64] = a0 * q[u].y + b0 * q[u].x;
+          v[i + 1] = a1 * q[u].z - b1 * q[u].w;
+          v[i + 65] = a1 * q[u].w + b1 * q[u].z;
+        }
       }
     }
   }
@@ -364,6 +427,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const int G = static_cast<int>(gridDim.x >> 1);
   const int c = static_cast<int>(blockIdx.x >> 1);
 
+  // Programmatic dependent launch: the next kernel in the stream may start
+  // its own prologue once every CTA of this grid got here.
+  griddep_launch_dependents();
+
   if (warp == 0) {
     if (lane == 0) {
       int stage = 0;
@@ -372,25 +439,50 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       WorkIter it(p, c, G);
       Work w;
       bool ok = true;
-      while (ok && it.next(w)) {
+      bool have = it.next(w);
+      // The weights (B) do not depend on the previous kernel in the stream:
+      // the first stages' B boxes are requested before waiting for it, the A
+      // boxes (this layer's activations) after.
+      int pre = 0;
+      if (have) {
+        int64_t tm, tn;
+        tile_mn(p, w.tile, num_m, num_n, tm, tn);
+        const int32_t n0 = static_cast<int32_t>(tn * BN + rank * (BN / 2));
+        pre = w.kb1 - w.kb0 < S ? w.kb1 - w.kb0 : S;
+        for (int i = 0; i < pre; ++i) {
+          const uint32_t fb = map_to_cta(smem_u32(full + i), 0);
+          if (lead_cta) mbar_arrive_expect_tx(full + i, 2 * C::kStageBytes);
+          tma_load_2d_pair(smB + i * C::kBBytes, &tmB, fb, (w.kb0 + i) * BK, n0);
+        }
+      }
+      griddep_wait();
+      bool first = true;
+      while (ok && have) {
         int64_t tm, tn;
         tile_mn(p, w.tile, num_m, num_n, tm, tn);
         const int32_t m0 = static_cast<int32_t>(tm * 2 * BM + rank * BM);
         const int32_t n0 = static_cast<int32_t>(tn * BN + rank * (BN / 2));
         for (int kb = w.kb0; kb < w.kb1; ++kb) {
-          if (!mbar_wait(empty + stage, ph ^ 1, p.err, kWhereGemmProducer, abort_flag)) {
-            ok = false;
-            break;
-          }
-          // both CTAs' loads complete on the even CTA's barrier
           const uint32_t fb = map_to_cta(smem_u32(full + stage), 0);
-          if (lead_cta) mbar_arrive_expect_tx(full + stage, 2 * C::kStageBytes);
-          tma_load_2d_pair(smA + stage * C::kABytes, &tmA, fb, kb * BK, m0);
-          tma_load_2d_pair(smB + stage * C::kBBytes, &tmB, fb, kb * BK, n0);
+          if (first && kb - w.kb0 < pre) {
+            // B already requested; stage `stage` is in its first use
+            tma_load_2d_pair(smA + stage * C::kABytes, &tmA, fb, kb * BK, m0);
+          } else {
+            if (!mbar_wait(empty + stage, ph ^ 1, p.err, kWhereGemmProducer, abort_flag)) {
+              ok = false;
+              break;
+            }
+            // both CTAs' loads complete on the even CTA's barrier
+            if (lead_cta) mbar_arrive_expect_tx(full + stage, 2 * C::kStageBytes);
+            tma_load_2d_pair(smA + stage * C::kABytes, &tmA, fb, kb * BK, m0);
+            tma_load_2d_pair(smB + stage * C::kBBytes, &tmB, fb, kb * BK, n0);
+          }
           issued |= 1u << stage;
           last_ph = (last_ph & ~(1u << stage)) | (ph << stage);
           if (++stage == S) { stage = 0; ph ^= 1; }
         }
+        first = false;
+        have = ok && it.next(w);
       }
       // Every issued load must land before the pair exits (the even CTA's
       // barrier counts both CTAs' bytes; the final cluster barrier holds the
@@ -439,6 +531,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       mbar_wait(drain, 0, p.err, kWhereGemmDrain, nullptr);
     }
   } else {
+    griddep_wait();  // the epilogue reads and writes this layer's activations
     const int quarter = warp & 3;
     const int rr = quarter * 32 + lane;
     const bool el = warp == 2 && lane == 0;  // epilogue leader
@@ -488,20 +581,23 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       if (w.role == kContributor) {
         // leave this CTA's fp32 partial rows in its slot, then raise its flag
         float* slot = p.sk_partials + static_cast<size_t>(blockIdx.x) * slot_floats;
+        const bool slot_ok =
+            dcheck(static_cast<int>(blockIdx.x) < p.sk_slots, p.err, kWhereDbgGemmScratch);
 #pragma unroll 1
-        for (int cc = 0; cc < BN / 32; ++cc) {
+        for (int cc = 0; slot_ok && cc < BN / 32; ++cc) {
           uint32_t r[32];
           tmem_ld32(tbase + 32 * cc, r);
           tmem_ld_wait();
-          float4* dst = reinterpret_cast<float4*>(slot + (static_cast<size_t>(cc) * BM + rr) * 32);
+          float4* dst = reinterpret_cast<float4*>(slot);
 #pragma unroll
           for (int j = 0; j < 8; ++j)
-            __stcg(dst + j, make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                                        __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])));
+            __stcg(dst + part_f4(cc, j, rr),
+                   make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                               __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])));
         }
         __threadfence();
         epilogue_sync();
-        if (el) st_release(p.sk_flags + blockIdx.x, 1);
+        if (el && slot_ok) st_release(p.sk_flags + blockIdx.x, 1);
       } else {
         const float* part = nullptr;
         int n_part = 0;
@@ -509,12 +605,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         if (w.role == kFinisher) {
           // contributors: the pairs owning k-blocks [kb1, KB) of this tile
           const int64_t t_rel = w.tile - p.dp_tiles;
-          const int c_last = sk_owner((t_rel + 1) * p.kb_per_tile - 1, p.sk_units, G);
+          const int c_last = sk_owner((t_rel + 1) * p.kb_per_tile - 1, p.sk_units, p.sk_pairs);
           const int first = 2 * (c + 1) + static_cast<int>(rank);
           part = p.sk_partials + static_cast<size_t>(first) * slot_floats;
           n_part = c_last - c;
+          if (!dcheck(2 * c_last + static_cast<int>(rank) < p.sk_slots, p.err,
+                      kWhereDbgGemmScratch))
+            n_part = 0;
           if (el) {
-            for (int cp = c + 1; cp <= c_last; ++cp) {
+            for (int cp = c + 1; cp <= c + n_part; ++cp) {
               int32_t* flag = p.sk_flags + 2 * cp + rank;
               const uint64_t t0 = globaltimer_ns();
               while (ld_acquire(flag) != 1) {
@@ -531,26 +630,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           epilogue_sync();
         }
         if constexpr (EPI == static_cast<int>(Epi::kQkv)) {
+          const float s = valid ? row_inv_rms(p, row) : 0.f;
 #pragma unroll 1
           for (int hh = 0; hh < BN / 128; ++hh)
-            qkv_head<BN>(tbase + 128 * hh, 4 * hh, rr, part, n_part, slot_stride, row, valid,
+            qkv_head<BN>(tbase + 128 * hh, 4 * hh, rr, part, n_part, slot_stride, row, valid, s,
                          n0 + 128 * hh, p, tile);
         } else if constexpr (EPI == static_cast<int>(Epi::kSwiGLU)) {
-          float s = 0.f;
-          if (valid) {
-            if (p.rowsq_in != nullptr) {
-              float ss = 0.f;
-              for (int t = 0; t < p.rowsq_n; ++t) ss += p.rowsq_in[row * p.rowsq_n + t];
-              s = 1.0f / sqrtf(ss / p.rowsq_width + p.eps);
-            } else {
-              s = p.row_scale[row];
-            }
-          }
+          const float s = valid ? row_inv_rms(p, row) : 0.f;
 #pragma unroll 1
           for (int cc = 0; cc < 4; ++cc) {
             float g[32], u[32];
-            load_chunk<BN>(tbase + 32 * cc, cc, rr, part, n_part, slot_stride, g);
-            load_chunk<BN>(tbase + 128 + 32 * cc, cc + 4, rr, part, n_part, slot_stride, u);
+            load_chunk<BN, 2>(tbase + 32 * cc, cc, rr, part, n_part, slot_stride, g);
+            load_chunk<BN, 2>(tbase + 128 + 32 * cc, cc + 4, rr, part, n_part, slot_stride, u);
             float v[32];
 #pragma unroll
             for (int t = 0; t < 32; ++t) v[t] = silu_fast(g[t] * s) * (u[t] * s);
@@ -562,7 +653,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 #pragma unroll 1
           for (int cc = 0; cc < BN / 32; ++cc) {
             float v[32];
-            load_chunk<BN>(tbase + 32 * cc, cc, rr, part, n_part, slot_stride, v);
+            load_chunk<BN, 4>(tbase + 32 * cc, cc, rr, part, n_part, slot_stride, v);
             if constexpr (kRes) {
               add_staged_bf16x32(tile, rr, cc, v);
               if (dsk >= 0) add_bf16x32(v, p.ds_slab + int64_t(dsk) * p.N + n0 + 32 * cc);
@@ -570,7 +661,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             if (p.rowsq_out != nullptr) ss += stage_bf16x32_ss(tile, rr, cc, v);
             else stage_bf16x32(tile, rr, cc, v);
           }
-          if (p.rowsq_out != nullptr && valid) p.rowsq_out[row * p.rowsq_n + tn] = ss;
+          if (p.rowsq_out != nullptr && valid &&
+              dcheck(tn < p.rowsq_n, p.err, kWhereDbgGemmRowsq))
+            p.rowsq_out[row * p.rowsq_n + tn] = ss;
         }
         fence_proxy_async_smem();
       }
@@ -603,35 +696,41 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   }
 }
 
-// Host-side schedule over pair tiles: data-parallel waves, and stream-K over
-// the remainder when whole waves would leave many pairs idle.
+// Host-side schedule over pair tiles. Whole waves of tiles run data
+// parallel. The tiles of a last, partial wave (rem < G of them) are each
+// split along K into s = G / rem equal ranges (at most s_cap, and ranges of
+// at least 4 k-blocks) run by rem * s pairs (stream-K over exactly those
+// tiles), so that wave costs about 1/s of a tile instead of a whole one. Every pair of a wave starts its tiles at k-block 0 and moves
+// through K at the same pace, so the pairs running at one time read the same
+// k-slab of the operand panels and L2 serves the repeats. Problems smaller
+// than one wave split each tile into ranges of at least 8 k-blocks.
 struct HostSched {
   int pairs;
+  int sk_pairs;
   int64_t dp_tiles, sk_units;
 };
 
-HostSched make_sched(int64_t tiles, int kb, int max_pairs) {
+HostSched make_sched(int64_t tiles, int kb, int max_pairs, int s_cap) {
   HostSched h{};
-  const int64_t waves = (tiles + max_pairs - 1) / max_pairs;
-  const double dp_eff = static_cast<double>(tiles) / static_cast<double>(waves * max_pairs);
-  if (dp_eff >= 0.85) {
-    h.pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
+  const int64_t G = max_pairs;
+  const int64_t full = tiles / G, rem = tiles % G;
+  int64_t s = rem > 0 ? G / rem : 1;
+  const int64_t s_max = full == 0 ? kb / 8 : kb / 4;  // keep ranges a few k-blocks long
+  if (s > s_max) s = s_max;
+  if (s > s_cap) s = s_cap;
+  if (s < 1) s = 1;
+  if (rem == 0 || s == 1) {
+    // data parallel: whole tiles, round robin over the pairs
+    h.pairs = static_cast<int>(tiles < G ? tiles : G);
     h.dp_tiles = tiles;
     h.sk_units = 0;
+    h.sk_pairs = 1;
     return h;
   }
-  const int64_t full_waves = tiles / max_pairs;
-  h.dp_tiles = full_waves > 0 ? (full_waves - 1) * max_pairs : 0;
-  h.sk_units = (tiles - h.dp_tiles) * kb;
-  int64_t g = max_pairs;
-  if (tiles < max_pairs) {
-    // small problems: whole tiles, or at least 8 k-blocks per pair
-    const int64_t by_units = (h.sk_units + 7) / 8;
-    g = tiles > by_units ? tiles : by_units;
-    if (g > max_pairs) g = max_pairs;
-  }
-  if (g > h.sk_units) g = h.sk_units;
-  h.pairs = static_cast<int>(g);
+  h.dp_tiles = full * G;
+  h.sk_units = rem * kb;
+  h.sk_pairs = static_cast<int>(rem * s);
+  h.pairs = static_cast<int>(full > 0 ? G : h.sk_pairs);
   return h;
 }
 
@@ -650,24 +749,19 @@ cudaError_t launch_bn(const GemmArgs& a, Params p, cudaStream_t st) {
     tmRes = tmOut;
   }
   auto kern = gemm_tc_kernel<BN, EPI>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(C::kSmem));
+  cudaError_t e = smem_attr_at_least(reinterpret_cast<const void*>(kern), C::kSmem);
   if (e != cudaSuccess) return e;
   // Stream-K finishers wait on other pairs, so every pair of the grid must be
   // resident at once: the grid never exceeds the co-resident cluster count.
-  static int max_clusters = 0;
-  if (max_clusters == 0) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * (sm_count() / 2));
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = C::kSmem;
-    int n = 0;
-    e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
-    if (e != cudaSuccess) return e;
-    max_clusters = n > 0 ? (n < sm_count() / 2 ? n : sm_count() / 2) : 1;
-  }
+  int n = 0;
+  e = max_active_clusters(reinterpret_cast<const void*>(kern), kThreads, C::kSmem, 2, &n);
+  if (e != cudaSuccess) return e;
+  const int max_clusters = n > 0 ? (n < sm_count() / 2 ? n : sm_count() / 2) : 1;
   const int64_t tiles = ((a.M + 2 * BM - 1) / (2 * BM)) * (a.N / BN);
-  const HostSched h = make_sched(tiles, static_cast<int>(a.K / BK), max_clusters);
+  // The QKV finisher's epilogue (per-head norm and rotation over the summed
+  // partials) is the heaviest; more than two ranges per tile measured slower.
+  const int s_cap = EPI == static_cast<int>(Epi::kQkv) ? 2 : 1 << 20;
+  const HostSched h = make_sched(tiles, static_cast<int>(a.K / BK), max_clusters, s_cap);
   const int grid = 2 * h.pairs;
   if (h.sk_units > 0 &&
       (a.sk_partials == nullptr || a.sk_flags == nullptr || grid > a.sk_slots ||
@@ -675,10 +769,12 @@ cudaError_t launch_bn(const GemmArgs& a, Params p, cudaStream_t st) {
     return cudaErrorInvalidValue;
   p.dp_tiles = h.dp_tiles;
   p.sk_units = h.sk_units;
+  p.sk_pairs = h.sk_pairs;
   p.kb_per_tile = static_cast<int>(a.K / BK);
   // keep the smaller operand resident in L2 while the larger one streams
   p.m_fastest = a.M <= a.N ? 1 : 0;
-  kern<<<grid, kThreads, C::kSmem, st>>>(tmA, tmB, tmOut, tmRes, p);
+  e = launch_pdl_plain(kern, dim3(grid), dim3(kThreads), C::kSmem, st, tmA, tmB, tmOut, tmRes, p);
+  if (e != cudaSuccess) return e;
   return counted_launch(1);
 }
 
@@ -696,6 +792,7 @@ cudaError_t launch_gemm_tc(Epi epi, const GemmArgs& a, cudaStream_t st) {
   p.err = device_error_ptr();
   p.sk_partials = a.sk_partials;
   p.sk_flags = a.sk_flags;
+  p.sk_slots = a.sk_slots;
   p.rowsq_out = a.rowsq_out;
   p.rowsq_in = a.rowsq_in;
   p.rowsq_n = a.rowsq_n;

@@ -22,12 +22,36 @@ enum WhereTag : int32_t {
   kWherePositions = 301, kWhereDeepstackMap = 302, kWhereEmbed = 303, kWhereSelftest = 401,
   kWhereDecodeProducer = 501, kWhereDecodeMma = 502, kWhereDecodeEpilogue = 503,
   kWhereDecodeRange = 504, kWhereDecodeAttn = 505,
+  // bounds checks of the debug build (-DQ3VL_DEBUG)
+  kWhereDbgAttnStore = 601, kWhereDbgGemmScratch = 602, kWhereDbgGemmRowsq = 603,
+  kWhereDbgPositions = 604, kWhereDbgTable = 605, kWhereDbgRowstat = 606,
+  kWhereDbgDecodeStore = 607,
 };
 
 // Error record: [0] = status code, [1] = location tag. First error wins.
 __device__ __forceinline__ void record_error(int32_t* err, int32_t code, int32_t where) {
   if (err == nullptr) return;
   if (atomicCAS(err, 0, code) == 0) atomicExch(err + 1, where);
+}
+
+// Debug builds (-DQ3VL_DEBUG, libq3vl_debug.so) check the computed index of
+// every global access that the kernels do not route through TMA (whose unit
+// clips out-of-range boxes itself): a failed check records Q3VL_ERANGE with
+// its location tag and the access is skipped. In release builds the check is
+// the constant true and compiles away. This stands in for a device memory
+// checker, which is not used on this hardware.
+#ifdef Q3VL_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+__device__ __forceinline__ bool dcheck(bool ok, int32_t* err, int32_t where) {
+  if constexpr (kDebugChecks) {
+    if (!ok) record_error(err, Q3VL_ERANGE, where);
+    return ok;
+  } else {
+    return true;
+  }
 }
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {

@@ -8,6 +8,7 @@
 #include <stdint.h>
 
 #include <string>
+#include <utility>
 
 #include "q3vl.h"
 
@@ -26,7 +27,7 @@ inline size_t elem_bytes(const q3vl_config& c) { return c.dtype == Q3VL_DTYPE_BF
 
 // Offsets (bytes) of every region of the layer workspace.
 struct WsLayout {
-  size_t cos_sin = 0;  // fp32 [S][64][2]
+  size_t cos_sin = 0;  // fp32 cos/sin table: [S][64][2] (fp32 layers), slot-major (bf16)
   size_t inv1 = 0;     // fp32 [S] input-norm inv_rms
   size_t inv2 = 0;     // fp32 [S] post-attention-norm inv_rms
   size_t ds_map = 0;   // int32 [S]
@@ -68,6 +69,16 @@ cudaError_t launch_positions(const uint8_t* tt, int64_t S, const int32_t* grids,
                              int32_t* pos, int32_t* info, cudaStream_t st);
 cudaError_t launch_rope_table(const q3vl_config& c, const int32_t* pos, int64_t S, float* cs,
                               cudaStream_t st);
+// Converts a position-major cos/sin table ([S][64][2], the q3vl_rope_table
+// layout) into the slot-major one the bf16 QKV epilogue reads: float4
+// t * S + p = (cos, sin) of slots 2t, 2t + 1 at position p.
+cudaError_t launch_rope_slot_major(const float* cs, int64_t S, float* out, cudaStream_t st);
+// bf16 layer prologue in one launch: the cos/sin table (slot-major), the
+// input row statistic of x (skipped when x is NULL) and n_flags zeroed
+// stream-K flags.
+cudaError_t launch_layer_prologue(const q3vl_config& c, const int32_t* pos, int64_t S, float* cs,
+                                  const void* x, float* inv, int32_t* flags, int n_flags,
+                                  cudaStream_t st);
 cudaError_t launch_rowstat(const q3vl_config& c, const void* x, int64_t S, int64_t width,
                            float* inv, cudaStream_t st);
 cudaError_t launch_final_norm(const q3vl_config& c, void* x, int64_t S, const void* gain,
@@ -93,7 +104,8 @@ struct GemmArgs {
   const float* bias;       // [N] or null (kQkv)
   const float* q_norm;     // [128] (kQkv)
   const float* k_norm;     // [128] (kQkv)
-  const float* cos_sin;    // [M][64][2] (kQkv)
+  const float* cos_sin;    // (kQkv, bf16 path) slot-major: float4 t * M + r = (cos, sin) of
+                           // slots 2t, 2t + 1 at row r; (fp32 path) [M][64][2]
   int64_t q_cols, k_cols;  // column ranges [0,q_cols) = q heads, [q_cols, q_cols+k_cols) = k
   float eps;
   const void* resid;       // bf16 [M, ldo] (kResidual)
@@ -187,8 +199,41 @@ cudaError_t launch_kv_store(const q3vl_config& c, const void* qkv, int64_t S,
                             const q3vl_kv_cache& kv, int32_t seq, cudaStream_t st);
 cudaError_t launch_decode_advance(int B, int32_t* pos, int32_t* len, cudaStream_t st);
 
+// Launches `kernel` on `st` as a programmatic dependent of the kernel before
+// it in the stream (PDL): it may start while that kernel finishes, and must
+// call griddepcontrol.wait before it touches memory that kernel, or any
+// earlier one, reads or writes. Compile-time cluster dimensions of the kernel
+// apply as usual.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl_plain(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // Device count of SMs (cached per device).
 int sm_count();
+
+// Raises `kernel`'s dynamic shared-memory limit to at least `bytes` on the
+// current device. The attribute is set once per (kernel, device, size
+// increase), under a lock, so concurrent host threads never lower it under
+// one another.
+cudaError_t smem_attr_at_least(const void* kernel, size_t bytes);
+
+// Most clusters of `cluster` CTAs of `kernel` (with `threads` threads and
+// `smem` bytes of dynamic shared memory each) that the current device holds
+// at once; cached per (kernel, device) under a lock.
+cudaError_t max_active_clusters(const void* kernel, int threads, size_t smem, int cluster,
+                                int* out);
 
 // Adds n to the process-wide count of kernels this library enqueued and
 // returns the launch status of the last one.
