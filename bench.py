@@ -15,7 +15,7 @@ needed between steps.
             token types copied in, x' copied out, every step (uploads and
             downloads on their own streams, overlapping other steps' kernels);
   roofline  the dominant kernel (gate/up GEMM with SiLU*up epilogue), timed
-            live by stage events the library records inside every 4th timed
+            live by stage events the library records inside every 10th timed
             step (--stage-every); `kernels` has the same for every kernel;
   also      the 2B-shape layer, the 2B 28-layer stack and the 32B-shape
             50-layer encoder (S = 1064 and 8192), with the final-norm pass;
@@ -62,7 +62,7 @@ def parse():
     ap.add_argument("--workload", default=syn.Q4B_LAYER.name, choices=sorted(syn.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--stage-every", type=int, default=4,
+    ap.add_argument("--stage-every", type=int, default=10,
                     help="record the per-kernel stage events on every n-th timed step")
     ap.add_argument("--no-stacks", action="store_true",
                     help="skip the 2B 28-layer stack and 32B 50-layer encoder measurements")

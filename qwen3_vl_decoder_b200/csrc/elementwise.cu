@@ -305,11 +305,10 @@ cudaError_t launch_rope_slot_major(const float* cs, int64_t S, float* out, cudaS
 }
 
 // ---------------------------------------------------------------------------
-// The bf16 layer's prologue in one launch: P1 (the cos/sin table, written
-// slot-major as above) in blocks
-// [0, table_blocks), P2 (the input row statistic, a warp per row) in the
-// blocks after them, and the stream-K flags of the GEMMs set to zero by
-// block 0. Launched as a programmatic dependent: it waits for the previous
+// The bf16 layer's prologue in one launch: P2 (the input row statistic, a
+// warp per row) in the first blocks, P1 (the cos/sin table, written
+// slot-major as above) in the last table_blocks blocks, and the stream-K
+// flags of the GEMMs set to zero by the first table block. Launched as a programmatic dependent: it waits for the previous
 // kernel in the stream (the positions, or the previous layer) before reading
 // pos or x, and lets the QKV GEMM start its prologue early.
 // ---------------------------------------------------------------------------
@@ -320,14 +319,18 @@ layer_prologue_kernel(const int32_t* __restrict__ pos, int64_t S, double theta, 
                       float* __restrict__ inv, int32_t* __restrict__ flags, int n_flags) {
   griddep_wait();
   griddep_launch_dependents();
-  if (static_cast<int>(blockIdx.x) < table_blocks) {
+  // the row-statistic blocks come first, so the 21 MB pass over x starts at
+  // once on every SM and the table blocks fill in behind it
+  const int stat_blocks = static_cast<int>(gridDim.x) - table_blocks;
+  if (static_cast<int>(blockIdx.x) >= stat_blocks) {
+    const int tb = static_cast<int>(blockIdx.x) - stat_blocks;
     __shared__ double freq[kHalf];
     if (threadIdx.x < kHalf) freq[threadIdx.x] = pow(theta, -2.0 * threadIdx.x / kHeadDim);
-    if (blockIdx.x == 0)
+    if (tb == 0)
       for (int i = threadIdx.x; i < n_flags; i += blockDim.x) flags[i] = 0;
     __syncthreads();
     // slot-major: consecutive threads take consecutive positions of one slot
-    const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t idx = int64_t(tb) * blockDim.x + threadIdx.x;
     if (idx >= S * kHalf) return;
     const int i = static_cast<int>(idx / S);
     const int64_t pp = idx % S;
@@ -342,7 +345,7 @@ layer_prologue_kernel(const int32_t* __restrict__ pos, int64_t S, double theta, 
     return;
   }
   if (x == nullptr) return;
-  const int64_t row = int64_t(blockIdx.x - table_blocks) * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int64_t row = int64_t(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= S) return;
   const float sq = row_sumsq<__nv_bfloat16>(reinterpret_cast<const uint4*>(x + row * width),
