@@ -394,6 +394,16 @@ constexpr float kRescaleLog2 = 8.0f;
 // (more spill under the 168-register cap of a 320-thread CTA).
 constexpr int kPolyPairs = 4;
 
+// Persistent: one CTA per SM walks work items (query tile qt, head pair h0);
+// item k has qt = num_qt - 1 - k / pairs, so items come longest first, and
+// CTA c takes items c, 2G-1-c, 2G+c, 4G-1-c, ... (G CTAs, a snake that
+// evens out the causal tile counts). Across items the pipeline keeps going:
+// the TMA warp loads the next item's Q as soon as the last S of the current
+// item has read Q, the MMA warp issues the next item's first S products right
+// behind the current item's last P V, and only the next item's first P V
+// waits for the softmax warps to have read the finished O out of TMEM.
+// Barrier phases run on counters across items: per CTA item index ii and
+// per CTA tile index t (a tile = one key tile of one item).
 template <int kPoly>
 __global__ void __launch_bounds__(kThreads2, 1)
 attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
@@ -412,22 +422,29 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
   uint64_t* p_full = bars + 11;  // [2] per head
   uint64_t* o_final = bars + 13;
   uint64_t* drain = bars + 14;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+  uint64_t* q_empty = bars + 15;
+  uint64_t* o_free = bars + 16;  // [2] per head
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pairs = p.nh / 2;
-  const int qt = p.num_qt - 1 - static_cast<int>(blockIdx.x / pairs);
-  const int h0 = 2 * static_cast<int>(blockIdx.x % pairs);
-  const int g = h0 / (p.nh / p.nkv);
-  const int n_kv = qt + 1;
+  const int n_items = p.num_qt * pairs;
+  const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+  // the ii-th item of this CTA, or -1 past the end
+  auto item_of = [&](int ii) -> int {
+    const int k = (ii >> 1) * 2 * G + ((ii & 1) ? 2 * G - 1 - c : c);
+    return k < n_items ? k : -1;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(k_full + s, 1); mbar_init(k_empty + s, 1);
       mbar_init(v_full + s, 1); mbar_init(v_empty + s, 1);
       mbar_init(s_full + s, 1); mbar_init(p_full + s, 128);
+      mbar_init(o_free + s, 128);
     }
     mbar_init(o_final, 1);
     mbar_init(drain, 1);
@@ -450,42 +467,53 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
   if (warp == 0) {
     if (lane == 0) {
       griddep_wait();
-      mbar_arrive_expect_tx(q_full, 2 * kTileBytes);
-      for (int x = 0; x < 2; ++x) {
-        tma_load_2d(sQ + x * kTileBytes, &tm, q_full, (h0 + x) * 128, qt * kTile);
-        tma_load_2d(sQ + x * kTileBytes + kBlockBytes, &tm, q_full, (h0 + x) * 128 + 64,
-                    qt * kTile);
+      int nk_issued = 0, nv_issued = 0, nq_issued = 0;
+      bool ok = true;
+      for (int ii = 0, k = item_of(0); ok && k >= 0; k = item_of(++ii)) {
+        const int qt = p.num_qt - 1 - k / pairs, h0 = 2 * (k % pairs);
+        const int g = h0 / (p.nh / p.nkv);
+        // Q is free once the previous item's last S products completed
+        if (ii > 0 && !mbar_wait(q_empty, (ii - 1) & 1, p.err, kWhereAttnProducer, abort_flag)) break;
+        mbar_arrive_expect_tx(q_full, 2 * kTileBytes);
+        for (int x = 0; x < 2; ++x) {
+          tma_load_2d(sQ + x * kTileBytes, &tm, q_full, (h0 + x) * 128, qt * kTile);
+          tma_load_2d(sQ + x * kTileBytes + kBlockBytes, &tm, q_full, (h0 + x) * 128 + 64,
+                      qt * kTile);
+        }
+        ++nq_issued;
+        for (int j = 0; j <= qt; ++j) {
+          const int t = nk_issued, s = t & 1;
+          const uint32_t ph = (t >> 1) & 1;
+          if (!mbar_wait(k_empty + s, ph ^ 1, p.err, kWhereAttnProducer, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(k_full + s, kTileBytes);
+          tma_load_2d(sK + s * kTileBytes, &tm, k_full + s, p.k_col0 + g * 128, j * kTile);
+          tma_load_2d(sK + s * kTileBytes + kBlockBytes, &tm, k_full + s, p.k_col0 + g * 128 + 64,
+                      j * kTile);
+          ++nk_issued;
+          if (!mbar_wait(v_empty + s, ph ^ 1, p.err, kWhereAttnProducer, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(v_full + s, kTileBytes);
+          tma_load_2d(sV + s * kTileBytes, &tm, v_full + s, p.v_col0 + g * 128, j * kTile);
+          tma_load_2d(sV + s * kTileBytes + kBlockBytes, &tm, v_full + s, p.v_col0 + g * 128 + 64,
+                      j * kTile);
+          ++nv_issued;
+        }
       }
-      int nk_issued = 0, nv_issued = 0;
-      for (int j = 0; j < n_kv; ++j) {
-        const int s = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (!mbar_wait(k_empty + s, ph ^ 1, p.err, kWhereAttnProducer, abort_flag)) break;
-        mbar_arrive_expect_tx(k_full + s, kTileBytes);
-        tma_load_2d(sK + s * kTileBytes, &tm, k_full + s, p.k_col0 + g * 128, j * kTile);
-        tma_load_2d(sK + s * kTileBytes + kBlockBytes, &tm, k_full + s, p.k_col0 + g * 128 + 64,
-                    j * kTile);
-        ++nk_issued;
-        if (!mbar_wait(v_empty + s, ph ^ 1, p.err, kWhereAttnProducer, abort_flag)) break;
-        mbar_arrive_expect_tx(v_full + s, kTileBytes);
-        tma_load_2d(sV + s * kTileBytes, &tm, v_full + s, p.v_col0 + g * 128, j * kTile);
-        tma_load_2d(sV + s * kTileBytes + kBlockBytes, &tm, v_full + s, p.v_col0 + g * 128 + 64,
-                    j * kTile);
-        ++nv_issued;
-      }
-      mbar_wait(q_full, 0, p.err, kWhereAttnDrain, nullptr);
-      for (int j = nk_issued - 2; j < nk_issued; ++j)
-        if (j >= 0) mbar_wait(k_full + (j & 1), (j >> 1) & 1, p.err, kWhereAttnDrain, nullptr);
-      for (int j = nv_issued - 2; j < nv_issued; ++j)
-        if (j >= 0) mbar_wait(v_full + (j & 1), (j >> 1) & 1, p.err, kWhereAttnDrain, nullptr);
+      // every issued load lands before the block exits: the last Q and the
+      // last two loads of each ring are the only ones whose completion may be
+      // unseen
+      if (nq_issued > 0) mbar_wait(q_full, (nq_issued - 1) & 1, p.err, kWhereAttnDrain, nullptr);
+      for (int t = nk_issued - 2; t < nk_issued; ++t)
+        if (t >= 0) mbar_wait(k_full + (t & 1), (t >> 1) & 1, p.err, kWhereAttnDrain, nullptr);
+      for (int t = nv_issued - 2; t < nv_issued; ++t)
+        if (t >= 0) mbar_wait(v_full + (t & 1), (t >> 1) & 1, p.err, kWhereAttnDrain, nullptr);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, 128, false, true);
-      auto issue_s = [&](int x, int j) {
+      auto issue_s = [&](int x, int t) {
         const uint32_t q0 = smem_u32(sQ + x * kTileBytes);
-        const uint32_t k0 = smem_u32(sK + (j & 1) * kTileBytes);
+        const uint32_t k0 = smem_u32(sK + (t & 1) * kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * kBlockBytes + (kk & 3) * 32;
@@ -494,44 +522,62 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
         }
         umma_commit(s_full + x);
       };
-      auto issue_pv = [&](int x, int j) {
-        const uint32_t v0 = smem_u32(sV + (j & 1) * kTileBytes);
+      auto issue_pv = [&](int x, int j, int t) {
+        const uint32_t v0 = smem_u32(sV + (t & 1) * kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           umma_bf16_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8,
                        sdesc_sw128(v0 + kk * 2048, kBlockBytes, 1024), idesc_o, (j | kk) != 0);
       };
-      bool ok = mbar_wait(q_full, 0, p.err, kWhereAttnMma, abort_flag) &&
-                mbar_wait(k_full, 0, p.err, kWhereAttnMma, abort_flag);
-      if (ok) {
+      bool ok = true;
+      int t0 = 0;  // this CTA's tile index of the item's first key tile
+      for (int ii = 0, k = item_of(0); ok && k >= 0; k = item_of(++ii)) {
+        const int n_kv = p.num_qt - k / pairs;
+        ok = mbar_wait(q_full, ii & 1, p.err, kWhereAttnMma, abort_flag) &&
+             mbar_wait(k_full + (t0 & 1), (t0 >> 1) & 1, p.err, kWhereAttnMma, abort_flag);
+        if (!ok) break;
         tc_fence_after();
-        issue_s(0, 0);
-        issue_s(1, 0);
-        umma_commit(k_empty);
-      }
-      for (int j = 0; ok && j < n_kv; ++j) {
-        const int s = j & 1;
-        const bool more = j + 1 < n_kv;
-        if (!mbar_wait(v_full + s, (j >> 1) & 1, p.err, kWhereAttnMma, abort_flag)) break;
-        if (!mbar_wait(p_full + 0, j & 1, p.err, kWhereAttnMma, abort_flag)) break;
-        tc_fence_after();
-        issue_pv(0, j);
-        if (more) {
-          if (!mbar_wait(k_full + (s ^ 1), ((j + 1) >> 1) & 1, p.err, kWhereAttnMma, abort_flag))
-            break;
+        // S_X(0) overwrites P_X of the previous item's last tile only after
+        // that tile's P V, issued before it, has read it (in-order execution)
+        issue_s(0, t0);
+        issue_s(1, t0);
+        umma_commit(k_empty + (t0 & 1));
+        if (n_kv == 1) umma_commit(q_empty);
+        for (int j = 0; j < n_kv; ++j) {
+          const int t = t0 + j, s = t & 1;
+          const bool more = j + 1 < n_kv;
+          if (!mbar_wait(v_full + s, (t >> 1) & 1, p.err, kWhereAttnMma, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(p_full + 0, t & 1, p.err, kWhereAttnMma, abort_flag)) { ok = false; break; }
+          // the first P V of an item overwrites O: the previous item's O_A
+          // must have been read out
+          if (j == 0 && ii > 0 &&
+              !mbar_wait(o_free + 0, (ii - 1) & 1, p.err, kWhereAttnMma, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          issue_s(0, j + 1);
+          issue_pv(0, j, t);
+          if (more) {
+            if (!mbar_wait(k_full + (s ^ 1), ((t + 1) >> 1) & 1, p.err, kWhereAttnMma, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_s(0, t + 1);
+          }
+          if (!mbar_wait(p_full + 1, t & 1, p.err, kWhereAttnMma, abort_flag)) { ok = false; break; }
+          if (j == 0 && ii > 0 &&
+              !mbar_wait(o_free + 1, (ii - 1) & 1, p.err, kWhereAttnMma, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(1, j, t);
+          umma_commit(v_empty + s);
+          if (more) {
+            issue_s(1, t + 1);
+            umma_commit(k_empty + (s ^ 1));
+            if (j + 2 == n_kv) umma_commit(q_empty);  // the item's last S products
+          }
         }
-        if (!mbar_wait(p_full + 1, j & 1, p.err, kWhereAttnMma, abort_flag)) break;
-        tc_fence_after();
-        issue_pv(1, j);
-        umma_commit(v_empty + s);
-        if (more) {
-          issue_s(1, j + 1);
-          umma_commit(k_empty + (s ^ 1));
-        }
+        umma_commit(o_final);
+        t0 += n_kv;
       }
-      umma_commit(o_final);
+      if (!ok) *abort_flag = 1;
       umma_commit(drain);
       mbar_wait(drain, 0, p.err, kWhereAttnDrain, nullptr);
     }
@@ -542,69 +588,74 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
     const uint32_t lane_field = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tmem + x * 128 + lane_field;
     const uint32_t tO = tmem + 256 + x * 128 + lane_field;
-    const int64_t qpos = int64_t(qt) * kTile + r;
     const float sc = p.scale_log2;
-    float m = -INFINITY, l = 0.f;
+    griddep_wait();  // before this kernel's global stores
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      ok = mbar_wait(s_full + x, j & 1, p.err, kWhereAttnSoftmax, abort_flag);
+    int t = 0;  // this CTA's running tile index
+    for (int ii = 0, k = item_of(0); ok && k >= 0; k = item_of(++ii)) {
+      const int qt = p.num_qt - 1 - k / pairs, h0 = 2 * (k % pairs);
+      const int64_t qpos = int64_t(qt) * kTile + r;
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j <= qt; ++j, ++t) {
+        ok = mbar_wait(s_full + x, t & 1, p.err, kWhereAttnSoftmax, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        tc_fence_after();
+        const bool diag = j == qt;
+        // the whole score row in registers: one batch of TMEM loads, one wait
+        uint32_t sr[128];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) tmem_ld32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(sr + 32 * cc));
+        tmem_ld_wait();
+        // row max of the raw (unscaled) scores; the scale is positive
+        const float mx = diag ? row_max_regs<true>(sr, r) : row_max_regs<false>(sr, r);
+        const float m_new = fmaxf(m, mx * sc);
+        const bool grow = m_new > m + kRescaleLog2;
+        const float alpha = grow ? ex2_approx(m - m_new) : 1.0f;
+        if (grow) m = m_new;
+        // P = 2^(s*scale - m) as bf16 into the first 64 columns of S
+        const float rs = diag ? exp_regs<true, kPoly>(sr, tS, r, sc, m)
+                              : exp_regs<false, kPoly>(sr, tS, r, sc, m);
+        l = l * alpha + rs;
+        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+          // O_X(j-1) is complete: S_X(j) was issued after P_X(j-1) V(j-1).
+#pragma unroll 1
+          for (int c4 = 0; c4 < 4; ++c4) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * c4, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int u = 0; u < 32; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
+            tmem_st32(tO + 32 * c4, o);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(p_full + x);
+      }
+      if (!ok) break;
+      ok = mbar_wait(o_final, ii & 1, p.err, kWhereAttnSoftmax, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      const bool diag = j == qt;
-      // the whole score row in registers: one batch of TMEM loads, one wait
-      uint32_t sr[128];
+      const float inv_l = 1.0f / l;
+      __nv_bfloat16* dst = p.o + qpos * p.ldo + (h0 + x) * 128;
+      uint32_t o[4][32];
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) tmem_ld32(tS + 32 * cc, *reinterpret_cast<uint32_t(*)[32]>(sr + 32 * cc));
+      for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tO + 32 * c4, o[c4]);
       tmem_ld_wait();
-      // row max of the raw (unscaled) scores; the scale is positive
-      const float mx = diag ? row_max_regs<true>(sr, r) : row_max_regs<false>(sr, r);
-      const float m_new = fmaxf(m, mx * sc);
-      const bool grow = m_new > m + kRescaleLog2;
-      const float m_use = grow ? m_new : m;
-      const float alpha = grow ? ex2_approx(m - m_new) : 1.0f;
-      // P = 2^(s*scale - m) as bf16 into the first 64 columns of S
-      const float rs = diag ? exp_regs<true, kPoly>(sr, tS, r, sc, m_use)
-                            : exp_regs<false, kPoly>(sr, tS, r, sc, m_use);
-      l = l * alpha + rs;
-      m = m_use;
-      if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        // O_X(j-1) is complete: S_X(j) was issued after P_X(j-1) V(j-1).
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + 32 * c, o);
-          tmem_ld_wait();
-#pragma unroll
-          for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * alpha);
-          tmem_st32(tO + 32 * c, o);
-        }
-      }
-      tmem_st_wait();
+      // O is in registers: the next item's first P V may overwrite it
       tc_fence_before();
-      mbar_arrive(p_full + x);
-    }
-    griddep_wait();  // before this kernel's global stores
-    if (ok) {
-      ok = mbar_wait(o_final, 0, p.err, kWhereAttnSoftmax, abort_flag);
-      if (__all_sync(0xffffffffu, ok)) {
-        tc_fence_after();
-        const float inv_l = 1.0f / l;
-        __nv_bfloat16* dst = p.o + qpos * p.ldo + (h0 + x) * 128;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + 32 * c, o);
-          tmem_ld_wait();
-          if (qpos < p.S && dcheck(((h0 + x) + 1) * 128 <= p.ldo, p.err, kWhereDbgAttnStore)) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+      mbar_arrive(o_free + x);
+      if (qpos < p.S && dcheck(((h0 + x) + 1) * 128 <= p.ldo, p.err, kWhereDbgAttnStore)) {
 #pragma unroll
-            for (int t = 0; t < 4; ++t)
-              d4[t] = make_uint4(
-                  pack_bf16x2(__uint_as_float(o[8 * t]) * inv_l, __uint_as_float(o[8 * t + 1]) * inv_l),
-                  pack_bf16x2(__uint_as_float(o[8 * t + 2]) * inv_l, __uint_as_float(o[8 * t + 3]) * inv_l),
-                  pack_bf16x2(__uint_as_float(o[8 * t + 4]) * inv_l, __uint_as_float(o[8 * t + 5]) * inv_l),
-                  pack_bf16x2(__uint_as_float(o[8 * t + 6]) * inv_l, __uint_as_float(o[8 * t + 7]) * inv_l));
-          }
+        for (int c4 = 0; c4 < 4; ++c4) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c4);
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            d4[u] = make_uint4(
+                pack_bf16x2(__uint_as_float(o[c4][8 * u]) * inv_l, __uint_as_float(o[c4][8 * u + 1]) * inv_l),
+                pack_bf16x2(__uint_as_float(o[c4][8 * u + 2]) * inv_l, __uint_as_float(o[c4][8 * u + 3]) * inv_l),
+                pack_bf16x2(__uint_as_float(o[c4][8 * u + 4]) * inv_l, __uint_as_float(o[c4][8 * u + 5]) * inv_l),
+                pack_bf16x2(__uint_as_float(o[c4][8 * u + 6]) * inv_l, __uint_as_float(o[c4][8 * u + 7]) * inv_l));
         }
       }
     }
@@ -640,7 +691,8 @@ cudaError_t launch_attention_tc(const q3vl_config& c, const void* qkv, int64_t S
     auto kern = attn2_tc_kernel<kPolyPairs>;
     cudaError_t e = smem_attr_at_least(reinterpret_cast<const void*>(kern), kSmem2);
     if (e != cudaSuccess) return e;
-    const unsigned grid = static_cast<unsigned>(int64_t(p.num_qt) * (p.nh / 2));
+    const int64_t items = int64_t(p.num_qt) * (p.nh / 2);
+    const unsigned grid = static_cast<unsigned>(items < sm_count() ? items : sm_count());
     e = launch_pdl_plain(kern, dim3(grid), dim3(kThreads2), kSmem2, st, tm, p);
     if (e != cudaSuccess) return e;
     return counted_launch(1);
