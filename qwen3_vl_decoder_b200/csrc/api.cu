@@ -69,6 +69,20 @@ cudaError_t smem_attr_at_least(const void* kernel, size_t bytes) {
   return e;
 }
 
+cudaError_t allow_nonportable_clusters(const void* kernel) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, bool> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(mu);
+  bool& d = done[{kernel, dev}];
+  if (d) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess) d = true;
+  return e;
+}
+
 cudaError_t max_active_clusters(const void* kernel, int threads, size_t smem, int cluster,
                                 int* out) {
   static std::mutex mu;

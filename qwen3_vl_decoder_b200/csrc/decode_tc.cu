@@ -384,6 +384,8 @@ constexpr int kAttnSmall = 16 * 64 * 2;    // one [16 rows x 64] bf16 swizzle bl
 
 struct DecAttnTcParams {
   const __nv_bfloat16* q;        // [B][nh*128]
+  const __nv_bfloat16* kc;       // the caches [n_seq][cap][nkv*128]
+  const __nv_bfloat16* vc;
   int64_t cap;
   int n_seq;
   const int32_t* seq;
@@ -396,7 +398,11 @@ struct DecAttnTcParams {
   uint32_t* tickets;             // [B][nkv], zero between launches
   int32_t* err;
   int nsplit;                    // most splits of one (b, g); nc_pad = nsplit rounded up to 4
+  int nbuf;                      // K/V stages in shared memory (1 .. kAttnMaxBuf)
+  int cs;                        // > 0: the nsplit = cs splits of a (b, g) form one cluster
 };
+
+constexpr int kAttnMaxBuf = 3;
 
 // Byte offset of element (row r, column c) in a 128-byte-swizzled tile of
 // 64-column blocks with `block_bytes` per block (rows of 128 bytes).
@@ -407,24 +413,29 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int c, uint32_t block_bytes
 }
 
 template <int G>
-__host__ __device__ constexpr size_t attn_tc_smem_bytes(int nc_pad) {
-  return 1024 + size_t(kAttnKV) + 2 * kAttnSmall +               // K/V, Q (P aliases Q)
+__host__ __device__ constexpr size_t attn_tc_smem_bytes(int nc_pad, int nbuf) {
+  return 1024 + size_t(nbuf) * kAttnKV + 2 * kAttnSmall +        // K/V stages, Q
+         (nbuf > 1 ? size_t(nbuf) * 2 * kAttnSmall : 0) +         // P (aliases Q if nbuf = 1)
          size_t(2) * G * nc_pad * 4 + size_t(4) * 8 * 4 * 2 +   // merge weights; warp partials
-         size_t(3) * G * 4 + (2 * kDecMaxB + 2) * 4 + 64;       // m, l, den; items; barriers
+         size_t(3) * G * 4 + (2 * kDecMaxB + 2) * 4 +           // m, l, den; items
+         size_t(G) * kAttnRows * 4 + 128;                        // cluster partial; barriers
 }
 
-template <int G>
+// NBUF (= p.nbuf) K/V stages: 1 for three CTAs per SM, kAttnMaxBuf for one.
+template <int G, int NBUF>
 __global__ void __launch_bounds__(kTcThreads, 3)
 decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, DecAttnTcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-  uint8_t* s_kv = sm;                                      // K0 K1 V0 V1
-  uint8_t* s_q = s_kv + kAttnKV;                           // [16 x 128] as 2 blocks
-  // P^T [16 x 128] reuses Q's tile: Q's reader (the S MMA) completed before P
-  // is written, and P's reader (the O MMA) before the next chunk writes Q
-  uint8_t* s_pt = s_q;
-  float* s_w = reinterpret_cast<float*>(s_q + 2 * kAttnSmall);  // [G][nc_pad]
+  uint8_t* s_kv = sm;                                      // [nbuf] x (K0 K1 V0 V1)
+  uint8_t* s_q = s_kv + size_t(NBUF) * kAttnKV;            // [16 x 128] as 2 blocks
+  // P^T [16 x 128] per chunk of a batch. With one stage it reuses Q's tile
+  // (Q's reader, the S MMA, completed before P is written, and P's reader,
+  // the O MMA, before the next chunk rewrites Q).
+  constexpr bool alias_q = NBUF == 1;
+  uint8_t* s_pt = alias_q ? s_q : s_q + 2 * kAttnSmall;   // [nbuf] tiles
+  float* s_w = reinterpret_cast<float*>(s_q + 2 * kAttnSmall * (alias_q ? 1 : 1 + NBUF));  // [G][nc_pad]
   float* s_cl = s_w + G * p.nc_pad;                        // [G][nc_pad]
   float* s_wm = s_cl + G * p.nc_pad;                       // [4 warps][8]
   float* s_wl = s_wm + 32;                                 // [4 warps][8]
@@ -434,18 +445,21 @@ decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tmK,
   int* s_nc = reinterpret_cast<int*>(s_den + G);           // [kDecMaxB] splits per token
   int* s_pref = s_nc + kDecMaxB;                           // [kDecMaxB + 1]
   int* s_last = s_pref + kDecMaxB + 1;
+  float* s_part = reinterpret_cast<float*>(s_last + 1);    // [G][kAttnRows]: o[128], m, l
   uint64_t* bars = reinterpret_cast<uint64_t*>(
-      (reinterpret_cast<uintptr_t>(s_last + 1) + 7) & ~uintptr_t(7));
-  uint64_t* kv_full = bars;
-  uint64_t* s_full = bars + 1;
-  uint64_t* o_full = bars + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3);
+      (reinterpret_cast<uintptr_t>(s_part + G * kAttnRows) + 7) & ~uintptr_t(7));
+  uint64_t* kv_full = bars;                                // [kAttnMaxBuf]
+  uint64_t* s_full = bars + kAttnMaxBuf;
+  uint64_t* o_full = s_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int nh = G * p.nkv;
+  constexpr int nbuf = NBUF;
+  constexpr uint32_t kOcol = 16 * NBUF, kTmemCols = NBUF == 1 ? 32 : 64;
   if (t == 0) {
-    mbar_init(kv_full, 1);
+    for (int i = 0; i < kAttnMaxBuf; ++i) mbar_init(kv_full + i, 1);
     mbar_init(s_full, 1);
     mbar_init(o_full, 1);
     *s_abort = 0;
@@ -454,7 +468,7 @@ decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tmK,
     tma_prefetch_desc(&tmV);
   }
   if (warp == 0) {
-    tmem_alloc(tmem_slot, 32);   // S^T in columns 0..15, O^T in 16..31
+    tmem_alloc(tmem_slot, kTmemCols);  // S^T of batch chunk i in columns 16 i .., O^T at kOcol
     tmem_relinquish();
   }
   tc_fence_before();
@@ -463,15 +477,16 @@ decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tmK,
   const uint32_t tmem = *tmem_slot;
   const uint32_t lane_field = static_cast<uint32_t>(warp * 32) << 16;
 
-  griddep_wait();
   griddep_launch_dependents();
   // items: (token b, KV head g, split s of b's chunks); each split walks a
-  // contiguous range of 128-row chunks
+  // contiguous range of 128-row chunks. Lengths and slots are inputs of the
+  // decode call, not outputs of the kernel before this one. In cluster mode
+  // every token has cs splits (some may get no chunk) and CTA i is item i.
   for (int b = t; b < p.B; b += kTcThreads) {
     const int slot = p.seq[b], L = p.len[b];
     const bool ok = slot >= 0 && slot < p.n_seq && L >= 0 && static_cast<int64_t>(L) < p.cap;
     const int nc = ok ? (L + kAttnCH) / kAttnCH : 0;  // chunks of rows 0..L
-    s_nc[b] = nc < p.nsplit ? nc : p.nsplit;
+    s_nc[b] = p.cs > 0 ? p.cs : (nc < p.nsplit ? nc : p.nsplit);
   }
   __syncthreads();
   if (warp == 0) {
@@ -499,45 +514,81 @@ decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tmK,
   }
   __syncthreads();
   const int total = s_pref[p.B];
-
-  constexpr uint32_t idesc_s = idesc_bf16_f32(128, 16, false, false);
-  constexpr uint32_t idesc_o = idesc_bf16_f32(128, 16, true, false);
-  int k = 0;  // chunks this CTA has processed: the phase of all three barriers
-  for (int it = blockIdx.x; it < total; it += gridDim.x) {
-    // a wait that timed out anywhere in the block ends the walk for all
-    // threads (read after the previous chunk's last barrier, written before it)
-    if (*s_abort) break;
+  // the item `it`: token, KV head, split and its chunk range (empty for a
+  // token whose slot or length is out of range)
+  auto item = [&](int it, int& b, int& g, int& c0, int& c1, int& splits, int& sidx) {
     int lo = 0, hi = p.B - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
       if (s_pref[mid] <= it) lo = mid;
       else hi = mid - 1;
     }
-    const int b = lo;
-    const int splits = s_nc[b];
+    b = lo;
+    splits = s_nc[b];
     const int loc = it - s_pref[b];
-    const int g = loc / splits, s = loc % splits;
+    g = loc / splits;
+    sidx = loc % splits;
+    const int slot = p.seq[b], L = p.len[b];
+    const bool ok = slot >= 0 && slot < p.n_seq && L >= 0 && static_cast<int64_t>(L) < p.cap;
+    const int nc = ok ? (L + kAttnCH) / kAttnCH : 0;
+    c0 = static_cast<int>(int64_t(sidx) * nc / splits);
+    c1 = static_cast<int>(int64_t(sidx + 1) * nc / splits);
+  };
+  // Loads run ahead of the chunk being computed by up to nbuf chunks, along
+  // this CTA's sequence of (item, chunk); only thread 0 walks it.
+  int l_it = blockIdx.x, l_b = 0, l_g = 0, l_c = 0, l_c1 = 0, n_issued = 0;
+  auto loader_seek = [&]() {  // from (l_it, l_c) to the next chunk that exists
+    while (l_it < total && l_c >= l_c1) {
+      int sp, si, c0;
+      item(l_it, l_b, l_g, c0, l_c1, sp, si);
+      l_c = c0;
+      if (l_c >= l_c1) l_it += gridDim.x;
+    }
+  };
+  auto load_next = [&]() {
+    if (l_it >= total) return;
+    const int st = n_issued % nbuf;
+    uint8_t* dst = s_kv + size_t(st) * kAttnKV;
+    const int32_t y = static_cast<int32_t>(int64_t(p.seq[l_b]) * p.cap + int64_t(l_c) * kAttnCH);
+    mbar_arrive_expect_tx(kv_full + st, kAttnKV);
+    tma_load_2d(dst, &tmK, kv_full + st, l_g * 128, y);
+    tma_load_2d(dst + kAttnBlk, &tmK, kv_full + st, l_g * 128 + 64, y);
+    tma_load_2d(dst + 2 * kAttnBlk, &tmV, kv_full + st, l_g * 128, y);
+    tma_load_2d(dst + 3 * kAttnBlk, &tmV, kv_full + st, l_g * 128 + 64, y);
+    ++n_issued;
+    ++l_c;
+    if (l_c >= l_c1) {
+      l_it += gridDim.x;
+      loader_seek();
+    }
+  };
+  // The cached rows below len[b] were written before this decode call and
+  // do not change during it, so the first nbuf chunks are loaded before
+  // waiting for the QKV projection; row len[b] (this token's K/V, written
+  // by that projection) is patched in after the wait.
+  if (t == 0) {
+    loader_seek();
+    for (int i = 0; i < nbuf; ++i) load_next();
+  }
+  griddep_wait();
+
+  constexpr uint32_t idesc_s = idesc_bf16_f32(128, 16, false, false);
+  constexpr uint32_t idesc_o = idesc_bf16_f32(128, 16, true, false);
+  int k = 0;   // chunks this CTA has processed: the phase of the stage barriers
+  int bi = 0;  // batches this CTA has processed: the phase of s_full and o_full
+  for (int it = blockIdx.x; it < total; it += gridDim.x) {
+    // a wait that timed out anywhere in the block ends the walk for all
+    // threads (read after the previous chunk's last barrier, written before
+    // it); in cluster mode the one item still reaches both cluster barriers
+    if (*s_abort && p.cs == 0) break;
+    int b, g, c0, c1, splits, s;
+    item(it, b, g, c0, c1, splits, s);
     const int L1 = p.len[b] + 1;
-    const int nc = (L1 + kAttnCH - 1) / kAttnCH;
-    const int c0 = static_cast<int>(int64_t(s) * nc / splits);
-    const int c1 = static_cast<int>(int64_t(s + 1) * nc / splits);
     float m_run[G], l_run[G], o_run[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) { m_run[h] = -INFINITY; l_run[h] = 0.f; o_run[h] = 0.f; }
 
-    for (int c = c0; c < c1; ++c, ++k) {
-      if (*s_abort) break;
-      if (t == 0) {
-        // this chunk's rows; the buffer's readers (the previous chunk's MMAs)
-        // completed before the previous chunk's last barrier
-        const int32_t y = static_cast<int32_t>(int64_t(p.seq[b]) * p.cap + int64_t(c) * kAttnCH);
-        mbar_arrive_expect_tx(kv_full, kAttnKV);
-        tma_load_2d(s_kv, &tmK, kv_full, g * 128, y);
-        tma_load_2d(s_kv + kAttnBlk, &tmK, kv_full, g * 128 + 64, y);
-        tma_load_2d(s_kv + 2 * kAttnBlk, &tmV, kv_full, g * 128, y);
-        tma_load_2d(s_kv + 3 * kAttnBlk, &tmV, kv_full, g * 128 + 64, y);
-      }
-      const int n = min(kAttnCH, L1 - c * kAttnCH);
+    auto build_q = [&]() {
       // Q^T operand: rows h < G are the query heads of KV head g, rows G..15 zero
       for (int ch = t; ch < 16 * 16; ch += kTcThreads) {
         const int h = ch >> 4, cc = ch & 15;
@@ -547,45 +598,92 @@ decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                                               int64_t(g * G + h) * 128 + cc * 8);
         *reinterpret_cast<uint4*>(s_q + sw128_off(h, cc * 8, kAttnSmall)) = v;
       }
-      if (!mbar_wait(kv_full, k & 1, p.err, kWhereDecodeAttn, s_abort)) *s_abort = 1;
+    };
+    if (!alias_q) build_q();
+    // Chunks go through in batches of up to nbuf (the stages holding them):
+    // one S MMA per chunk, one softmax over all the batch's rows, one O MMA
+    // per chunk accumulating into O^T, so the batch pays the chain's latency
+    // once.
+    for (int c = c0; c < c1;) {
+      if (*s_abort) break;
+      const int nb = min(nbuf, c1 - c);
+      // row len[b]: this token's K and V, from the cache row the QKV
+      // projection wrote (read after the wait); it lies in chunk cn
+      const int cn = (L1 - 1) / kAttnCH, r_new = L1 - 1 - cn * kAttnCH;
+      const bool has_new = cn >= c && cn < c + nb;
+      uint4 kv_new = make_uint4(0, 0, 0, 0);
+      if (has_new && t < 32) {
+        const int64_t row = int64_t(p.seq[b]) * p.cap + (L1 - 1);
+        const __nv_bfloat16* src = (t < 16 ? p.kc : p.vc) + row * (int64_t(p.nkv) * 128) + g * 128;
+        kv_new = *reinterpret_cast<const uint4*>(src + (t & 15) * 8);
+      }
+      if (alias_q) build_q();
+      for (int i = 0; i < nb; ++i)
+        if (!mbar_wait(kv_full + (k + i) % nbuf, ((k + i) / nbuf) & 1, p.err, kWhereDecodeAttn,
+                       s_abort))
+          *s_abort = 1;
+      if (has_new && t < 32)
+        *reinterpret_cast<uint4*>(s_kv + size_t((k + cn - c) % nbuf) * kAttnKV +
+                                  (t < 16 ? 0 : 2 * kAttnBlk) +
+                                  sw128_off(r_new, (t & 15) * 8, kAttnBlk)) = kv_new;
       // rows past the sequence hold whatever the cache had: zero V there (P is
-      // zero there, but 0 * NaN would not be)
-      for (int ch = t; ch < (kAttnCH - n) * 16; ch += kTcThreads) {
-        const int r = n + (ch >> 4), cc = ch & 15;
-        *reinterpret_cast<uint4*>(s_kv + 2 * kAttnBlk + (cc >> 3) * kAttnBlk + r * 128 +
-                                  (cc & 7) * 16) = make_uint4(0, 0, 0, 0);
+      // zero there, but 0 * NaN would not be); only chunk cn can be partial
+      if (has_new) {
+        uint8_t* kvn = s_kv + size_t((k + cn - c) % nbuf) * kAttnKV;
+        for (int ch = t; ch < (kAttnCH - 1 - r_new) * 16; ch += kTcThreads) {
+          const int r = r_new + 1 + (ch >> 4), cc = ch & 15;
+          *reinterpret_cast<uint4*>(kvn + 2 * kAttnBlk + (cc >> 3) * kAttnBlk + r * 128 +
+                                    (cc & 7) * 16) = make_uint4(0, 0, 0, 0);
+        }
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncthreads();
       if (t == 0 && *s_abort == 0) {
         tc_fence_after();
-        const uint32_t k0 = smem_u32(s_kv), q0 = smem_u32(s_q);
+        const uint32_t q0 = smem_u32(s_q);
+        for (int i = 0; i < nb; ++i) {
+          const uint32_t k0 = smem_u32(s_kv + size_t((k + i) % nbuf) * kAttnKV);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_bf16_ss(tmem, sdesc_sw128(k0 + (kk >> 2) * kAttnBlk + (kk & 3) * 32, 16, 1024),
-                       sdesc_sw128(q0 + (kk >> 2) * kAttnSmall + (kk & 3) * 32, 16, 1024),
-                       idesc_s, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk)
+            umma_bf16_ss(tmem + 16 * i,
+                         sdesc_sw128(k0 + (kk >> 2) * kAttnBlk + (kk & 3) * 32, 16, 1024),
+                         sdesc_sw128(q0 + (kk >> 2) * kAttnSmall + (kk & 3) * 32, 16, 1024),
+                         idesc_s, kk > 0 ? 1u : 0u);
+        }
         umma_commit(s_full);
       }
-      // softmax over the chunk's rows: thread t holds row t's scores of every head
-      float sc[16];
+      // softmax over the batch's rows: thread t holds row t of every chunk,
+      // the scores of every head
+      float sc[NBUF][16];
       {
         bool w_ok = true;
-        if (lane == 0) w_ok = mbar_wait(s_full, k & 1, p.err, kWhereDecodeAttn, s_abort);
+        if (lane == 0) w_ok = mbar_wait(s_full, bi & 1, p.err, kWhereDecodeAttn, s_abort);
         w_ok = __shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0) != 0;
         if (!w_ok) *s_abort = 1;
         tc_fence_after();
-        uint32_t u[16];
-        tmem_ld16(tmem + lane_field, u);
-        tmem_ld_wait();
 #pragma unroll
-        for (int h = 0; h < 16; ++h)
-          sc[h] = t < n ? __uint_as_float(u[h]) * p.scale_log2 : -INFINITY;
+        for (int i = 0; i < NBUF; ++i) {
+          if (i < nb) {
+            uint32_t u[16];
+            tmem_ld16(tmem + lane_field + 16 * i, u);
+            tmem_ld_wait();
+            const bool valid = (c + i) * kAttnCH + t < L1;
+#pragma unroll
+            for (int h = 0; h < 16; ++h)
+              sc[i][h] = valid ? __uint_as_float(u[h]) * p.scale_log2 : -INFINITY;
+          } else {
+#pragma unroll
+            for (int h = 0; h < 16; ++h) sc[i][h] = -INFINITY;
+          }
+        }
       }
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float wm = warp_max(sc[h]);
+        float v = sc[0][h];
+#pragma unroll
+        for (int i = 1; i < NBUF; ++i) v = fmaxf(v, sc[i][h]);
+        const float wm = warp_max(v);
         if (lane == 0) s_wm[warp * 8 + h] = wm;
       }
       __syncthreads();
@@ -593,48 +691,68 @@ decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tmK,
 #pragma unroll
       for (int h = 0; h < G; ++h)
         mh[h] = fmaxf(fmaxf(s_wm[h], s_wm[8 + h]), fmaxf(s_wm[16 + h], s_wm[24 + h]));
-      float pr[G];
+#pragma unroll
+      for (int i = 0; i < NBUF; ++i) {
+        if (i < nb) {
+          float pr[G];
+#pragma unroll
+          for (int h = 0; h < G; ++h)
+            pr[h] = sc[i][h] == -INFINITY ? 0.f : ex2_approx(sc[i][h] - mh[h]);
+          // P^T operand of chunk i: row h, column t (zero for h >= G)
+          uint8_t* pt = s_pt + size_t(alias_q ? 0 : i) * 2 * kAttnSmall;
+#pragma unroll
+          for (int h = 0; h < 16; ++h) {
+            const __nv_bfloat16 v = __float2bfloat16_rn(h < G ? pr[h < G ? h : 0] : 0.f);
+            *reinterpret_cast<__nv_bfloat16*>(pt + sw128_off(h, t, kAttnSmall)) = v;
+          }
+#pragma unroll
+          for (int h = 0; h < G; ++h) sc[i][h] = pr[h];
+        }
+      }
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        pr[h] = t < n ? ex2_approx(sc[h] - mh[h]) : 0.f;
-        const float ws = warp_sum(pr[h]);
-        if (lane == 0) s_wl[warp * 8 + h] = ws;
-      }
-      // P^T operand: row h, column t (zero for h >= G)
+        float v = 0.f;
 #pragma unroll
-      for (int h = 0; h < 16; ++h) {
-        const __nv_bfloat16 v = __float2bfloat16_rn(h < G ? pr[h < G ? h : 0] : 0.f);
-        *reinterpret_cast<__nv_bfloat16*>(s_pt + sw128_off(h, t, kAttnSmall)) = v;
+        for (int i = 0; i < NBUF; ++i)
+          if (i < nb) v += sc[i][h];
+        const float ws = warp_sum(v);
+        if (lane == 0) s_wl[warp * 8 + h] = ws;
       }
       fence_proxy_async_smem();
       tc_fence_before();
       __syncthreads();
       if (t == 0 && *s_abort == 0) {
         tc_fence_after();
-        const uint32_t v0 = smem_u32(s_kv + 2 * kAttnBlk), p0 = smem_u32(s_pt);
+        for (int i = 0; i < nb; ++i) {
+          const uint32_t v0 = smem_u32(s_kv + size_t((k + i) % nbuf) * kAttnKV + 2 * kAttnBlk);
+          const uint32_t p0 = smem_u32(s_pt + size_t(alias_q ? 0 : i) * 2 * kAttnSmall);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_bf16_ss(tmem + 16, sdesc_sw128(v0 + kk * 2048, kAttnBlk, 1024),
-                       sdesc_sw128(p0 + (kk >> 2) * kAttnSmall + (kk & 3) * 32, 16, 1024),
-                       idesc_o, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk)
+            umma_bf16_ss(tmem + kOcol, sdesc_sw128(v0 + kk * 2048, kAttnBlk, 1024),
+                         sdesc_sw128(p0 + (kk >> 2) * kAttnSmall + (kk & 3) * 32, 16, 1024),
+                         idesc_o, (i | kk) > 0 ? 1u : 0u);
+        }
         umma_commit(o_full);
       }
       float acc[G];
       {
         bool w_ok = true;
-        if (lane == 0) w_ok = mbar_wait(o_full, k & 1, p.err, kWhereDecodeAttn, s_abort);
+        if (lane == 0) w_ok = mbar_wait(o_full, bi & 1, p.err, kWhereDecodeAttn, s_abort);
         w_ok = __shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0) != 0;
         if (!w_ok) *s_abort = 1;
         tc_fence_after();
         uint32_t u[16];
-        tmem_ld16(tmem + lane_field + 16, u);
+        tmem_ld16(tmem + lane_field + kOcol, u);
         tmem_ld_wait();
 #pragma unroll
         for (int h = 0; h < G; ++h) acc[h] = __uint_as_float(u[h]);
       }
       tc_fence_before();
-      __syncthreads();  // TMEM and the operand tiles are free for the next chunk
-      // merge the chunk into the split's running (m, l, o)
+      __syncthreads();  // TMEM and the batch's stages are free
+      // the stages go to the chunks nbuf ahead
+      if (t == 0 && *s_abort == 0)
+        for (int i = 0; i < nb; ++i) load_next();
+      // merge the batch into the split's running (m, l, o)
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         const float lj = s_wl[h] + s_wl[8 + h] + s_wl[16 + h] + s_wl[24 + h];
@@ -644,9 +762,55 @@ decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tmK,
         l_run[h] = l_run[h] * wa + lj * wb;
         m_run[h] = M;
       }
+      c += nb;
+      k += nb;
+      ++bi;
     }
-    if (*s_abort) break;
+    if (*s_abort && p.cs == 0) break;
     __nv_bfloat16* ob = p.o + int64_t(b) * nh * 128 + int64_t(g) * G * 128;
+    if (p.cs > 0) {
+      // Cluster merge: the cs CTAs of the cluster are the cs splits of
+      // (b, g). Each leaves (o, m, l) of every head in its shared memory;
+      // after a cluster barrier CTA r finishes outputs r*128 + t, r*128 +
+      // t + 128 cs, ... of the G*128, reading the cs partials over DSMEM in
+      // split order; a second barrier keeps every CTA's partial alive until
+      // all reads are done. Every CTA passes both barriers.
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        s_part[h * kAttnRows + t] = o_run[h];
+        if (t == 0) {
+          s_part[h * kAttnRows + 128] = m_run[h];
+          s_part[h * kAttnRows + 129] = l_run[h];
+        }
+      }
+      cluster_sync();
+      const int slot = p.seq[b], L = p.len[b];
+      const bool tok_ok = slot >= 0 && slot < p.n_seq && L >= 0 && static_cast<int64_t>(L) < p.cap;
+      if (tok_ok && *s_abort == 0) {
+        const uint32_t r = cluster_ctarank();
+        for (int idx = static_cast<int>(r) * 128 + t; idx < G * 128; idx += p.cs * 128) {
+          const int h = idx >> 7, d = idx & 127;
+          const uint32_t base = smem_u32(s_part + h * kAttnRows);
+          float M = -INFINITY;
+          for (int sp = 0; sp < p.cs; ++sp)
+            M = fmaxf(M, ld_dsmem_f32(map_to_cta(base + 128 * 4, static_cast<uint32_t>(sp))));
+          float num = 0.f, den = 0.f;
+          for (int sp = 0; sp < p.cs; ++sp) {
+            const uint32_t ra = map_to_cta(base, static_cast<uint32_t>(sp));
+            const float m = ld_dsmem_f32(ra + 128 * 4);
+            if (m == -INFINITY) continue;  // a split without chunks
+            const float w = ex2_approx(m - M);
+            num = fmaf(w, ld_dsmem_f32(ra + 4u * d), num);
+            den = fmaf(w, ld_dsmem_f32(ra + 129 * 4), den);
+          }
+          if (dcheck(int64_t(b) < p.B, p.err, kWhereDbgDecodeStore))
+            ob[h * 128 + d] = __float2bfloat16_rn(num / den);
+        }
+      }
+      cluster_sync();
+      if (*s_abort) break;
+      continue;
+    }
     float* pb = p.part + (size_t(b) * p.nkv + g) * G * kAttnRows * size_t(p.nc_pad);
     if (splits == 1) {
 #pragma unroll
@@ -716,15 +880,16 @@ decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tmK,
     }
     __syncthreads();  // shared buffers are reused by the next item
   }
-  // every issued K/V load landed: each chunk waits for its own before going on,
-  // except a chunk cut short by a timeout
-  if (t == 0 && k > 0)
-    mbar_wait(kv_full, (k - 1) & 1, p.err, kWhereDecodeAttn, nullptr);
+  // every issued K/V load lands before the block exits: the loads not yet
+  // waited for are those of the last min(nbuf, n_issued) stages
+  if (t == 0)
+    for (int i = n_issued - nbuf; i < n_issued; ++i)
+      if (i >= 0) mbar_wait(kv_full + i % nbuf, (i / nbuf) & 1, p.err, kWhereDecodeAttn, nullptr);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 32);
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -874,16 +1039,62 @@ cudaError_t launch_dec_epi(const DecGemmArgs& a, int R, cudaStream_t st) {
 }
 
 template <int G>
-cudaError_t launch_attn_tc_g(const CUtensorMap& tmK, const CUtensorMap& tmV,
-                             const DecAttnTcParams& p, int grid, cudaStream_t st) {
-  const size_t smem = attn_tc_smem_bytes<G>(p.nc_pad);
+cudaError_t launch_attn_tc_g(const CUtensorMap& tmK, const CUtensorMap& tmV, DecAttnTcParams p,
+                             int64_t groups, int64_t max_nc, cudaStream_t st) {
+  const void* fn = reinterpret_cast<const void*>(decode_attn_tc_kernel<G, kAttnMaxBuf>);
+  // With at least two SMs per (b, g) (small batches) the splits of a (b, g)
+  // form one cluster of cs <= 16 CTAs, one CTA per SM with kAttnMaxBuf K/V
+  // stages, and merge over DSMEM; cs is the largest size whose clusters are
+  // all resident at once. Otherwise three CTAs share an SM with one stage
+  // each, items fill the CTA slots, and the last split of a (b, g) to finish
+  // merges the partials from global memory; there, about one item per SM
+  // (measured faster than filling all three slots: fewer partials to merge,
+  // none at all from 148 (b, g) on). Never more splits than the chunks of
+  // the longest sequence.
   {
-    const cudaError_t e =
-        smem_attr_at_least(reinterpret_cast<const void*>(decode_attn_tc_kernel<G>), smem);
+    const cudaError_t e = allow_nonportable_clusters(fn);
     if (e != cudaSuccess) return e;
   }
-  const cudaError_t e = launch_pdl(decode_attn_tc_kernel<G>, dim3(grid), dim3(kTcThreads), smem,
-                                   st, 1, tmK, tmV, p);
+  int64_t cs = sm_count() / groups;
+  if (cs > 16) cs = 16;
+  if (cs > max_nc) cs = max_nc;
+  p.cs = 0;
+  for (; cs >= 2; --cs) {
+    const int nc_pad = static_cast<int>((cs + 3) / 4 * 4);
+    const size_t smem = attn_tc_smem_bytes<G>(nc_pad, kAttnMaxBuf);
+    cudaError_t e = smem_attr_at_least(fn, smem);
+    if (e != cudaSuccess) return e;
+    int clusters = 0;
+    e = max_active_clusters(fn, kTcThreads, smem, static_cast<int>(cs), &clusters);
+    if (e != cudaSuccess) return e;
+    if (clusters >= groups) {
+      p.cs = static_cast<int>(cs);
+      break;
+    }
+  }
+  int64_t nsplit;
+  if (p.cs > 0) {
+    nsplit = p.cs;
+    p.nbuf = kAttnMaxBuf;
+  } else {
+    nsplit = (int64_t(sm_count()) + groups - 1) / groups;
+    if (nsplit > max_nc) nsplit = max_nc;
+    if (nsplit < 1) nsplit = 1;
+    p.nbuf = 1;
+  }
+  p.nsplit = static_cast<int>(nsplit);
+  p.nc_pad = static_cast<int>((nsplit + 3) / 4 * 4);
+  const int64_t items = groups * nsplit;
+  const int64_t cap_grid = 3 * int64_t(sm_count());
+  const int grid = static_cast<int>(p.cs > 0 || items < cap_grid ? items : cap_grid);
+  const size_t smem = attn_tc_smem_bytes<G>(p.nc_pad, p.nbuf);
+  auto kern = p.nbuf == 1 ? decode_attn_tc_kernel<G, 1> : decode_attn_tc_kernel<G, kAttnMaxBuf>;
+  {
+    const cudaError_t e = smem_attr_at_least(reinterpret_cast<const void*>(kern), smem);
+    if (e != cudaSuccess) return e;
+  }
+  const cudaError_t e = launch_pdl(kern, dim3(grid), dim3(kTcThreads), smem, st,
+                                   p.cs > 1 ? p.cs : 1, tmK, tmV, p);
   if (e != cudaSuccess) return e;
   return counted_launch(1);
 }
@@ -911,31 +1122,20 @@ cudaError_t launch_decode_attention(const q3vl_config& c, const void* q, const q
     return cudaErrorInvalidValue;
   DecAttnTcParams t{};
   t.q = static_cast<const __nv_bfloat16*>(q);
+  t.kc = static_cast<const __nv_bfloat16*>(kv.k);
+  t.vc = static_cast<const __nv_bfloat16*>(kv.v);
   t.cap = kv.cap; t.n_seq = kv.n_seq; t.seq = seq; t.len = len;
   t.B = B; t.nkv = c.n_kv_heads;
-  // splits per (b, g): with fewer groups than SMs (small batches) about one
-  // item per SM, each a few chunks long, so that fewer partials reach the
-  // merge (measured faster); otherwise fill the three CTA slots per SM;
-  // never more than the chunks of the longest sequence
   const int64_t groups = int64_t(B) * c.n_kv_heads;
-  const int64_t slots = (groups < sm_count() ? 1 : 3) * int64_t(sm_count());
   const int64_t max_nc = (kv.cap + kAttnCH - 1) / kAttnCH;
-  int64_t nsplit = (slots + groups - 1) / groups;
-  if (nsplit > max_nc) nsplit = max_nc;
-  if (nsplit < 1) nsplit = 1;
-  t.nsplit = static_cast<int>(nsplit);
-  t.nc_pad = static_cast<int>((nsplit + 3) / 4 * 4);
   t.scale_log2 = static_cast<float>(1.4426950408889634 / 11.313708498984761);  // log2(e)/sqrt(128)
   t.o = static_cast<__nv_bfloat16*>(o);
   t.part = part; t.tickets = tickets; t.err = device_error_ptr();
-  const int64_t items = groups * nsplit;
-  const int64_t cap_grid = 3 * int64_t(sm_count());
-  const int grid = static_cast<int>(items < cap_grid ? items : cap_grid);
   switch (G) {
-    case 1: return launch_attn_tc_g<1>(tmK, tmV, t, grid, st);
-    case 2: return launch_attn_tc_g<2>(tmK, tmV, t, grid, st);
-    case 4: return launch_attn_tc_g<4>(tmK, tmV, t, grid, st);
-    case 8: return launch_attn_tc_g<8>(tmK, tmV, t, grid, st);
+    case 1: return launch_attn_tc_g<1>(tmK, tmV, t, groups, max_nc, st);
+    case 2: return launch_attn_tc_g<2>(tmK, tmV, t, groups, max_nc, st);
+    case 4: return launch_attn_tc_g<4>(tmK, tmV, t, groups, max_nc, st);
+    case 8: return launch_attn_tc_g<8>(tmK, tmV, t, groups, max_nc, st);
     default: return cudaErrorInvalidValue;
   }
 }

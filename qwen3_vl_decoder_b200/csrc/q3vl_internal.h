@@ -229,6 +229,10 @@ int sm_count();
 // one another.
 cudaError_t smem_attr_at_least(const void* kernel, size_t bytes);
 
+// Lets `kernel` launch with clusters of more than 8 CTAs on the current
+// device; set once per (kernel, device), under a lock.
+cudaError_t allow_nonportable_clusters(const void* kernel);
+
 // Most clusters of `cluster` CTAs of `kernel` (with `threads` threads and
 // `smem` bytes of dynamic shared memory each) that the current device holds
 // at once; cached per (kernel, device) under a lock.
