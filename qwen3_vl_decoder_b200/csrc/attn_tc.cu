@@ -296,24 +296,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
 // registers (diagonal tile: keys past the query row excluded).
 template <bool kDiag>
 __device__ __forceinline__ float row_max_regs(const uint32_t* sr, int r) {
-  float mx = -INFINITY;
-  if (kDiag) {
+  // eight independent partial maxima keep the dependency chains short; on
+  // the diagonal tile the columns past r enter as -inf
+  auto v = [&](int c) {
+    const float x = __uint_as_float(sr[c]);
+    return kDiag && c > r ? -INFINITY : x;
+  };
+  float pm[8];
 #pragma unroll
-    for (int c = 0; c < 128; ++c)
-      if (c <= r) mx = fmaxf(mx, __uint_as_float(sr[c]));
-  } else {
-    // eight independent partial maxima keep the dependency chains short
-    float pm[8];
+  for (int q = 0; q < 8; ++q) pm[q] = fmaxf(v(q), v(q + 8));
 #pragma unroll
-    for (int q = 0; q < 8; ++q) pm[q] = fmaxf(__uint_as_float(sr[q]), __uint_as_float(sr[q + 8]));
+  for (int c = 16; c < 128; c += 16)
 #pragma unroll
-    for (int c = 16; c < 128; c += 16)
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        pm[q] = fmax3(pm[q], __uint_as_float(sr[c + q]), __uint_as_float(sr[c + q + 8]));
-    mx = fmaxf(fmaxf(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5])), fmaxf(pm[6], pm[7]));
-  }
-  return mx;
+    for (int q = 0; q < 8; ++q) pm[q] = fmax3(pm[q], v(c + q), v(c + q + 8));
+  return fmaxf(fmaxf(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5])), fmaxf(pm[6], pm[7]));
 }
 
 // 2^x for a pair of fp32 values on the FMA pipe (the special-function unit
