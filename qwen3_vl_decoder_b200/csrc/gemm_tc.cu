@@ -698,9 +698,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 
 // Host-side schedule over pair tiles. Whole waves of tiles run data
 // parallel. The tiles of a last, partial wave (rem < G of them) are each
-// split along K into s = G / rem equal ranges (at most s_cap, and ranges of
-// at least 4 k-blocks) run by rem * s pairs (stream-K over exactly those
-// tiles), so that wave costs about 1/s of a tile instead of a whole one. Every pair of a wave starts its tiles at k-block 0 and moves
+// split along K into s = G / rem equal ranges (ranges of at least 16
+// k-blocks) run by rem * s pairs (stream-K over exactly those tiles), so
+// that wave costs about 1/s of a tile instead of a whole one. Longer ranges
+// mean fewer partials for the finisher to add. On the 4B layer this gives
+// QKV and gate/up 2 ways, the o-projection 4 and down 6; measured there, the
+// o-projection took 65.0 us at 4 ways against 67.2 at 6 and 66.9 at 3, down
+// 141.6 at 6 against 142.7 at 4, and QKV was slower above 2. Every pair of a wave starts its tiles at k-block 0 and moves
 // through K at the same pace, so the pairs running at one time read the same
 // k-slab of the operand panels and L2 serves the repeats. Problems smaller
 // than one wave split each tile into ranges of at least 8 k-blocks.
@@ -710,14 +714,13 @@ struct HostSched {
   int64_t dp_tiles, sk_units;
 };
 
-HostSched make_sched(int64_t tiles, int kb, int max_pairs, int s_cap) {
+HostSched make_sched(int64_t tiles, int kb, int max_pairs) {
   HostSched h{};
   const int64_t G = max_pairs;
   const int64_t full = tiles / G, rem = tiles % G;
   int64_t s = rem > 0 ? G / rem : 1;
-  const int64_t s_max = full == 0 ? kb / 8 : kb / 4;  // keep ranges a few k-blocks long
+  const int64_t s_max = full == 0 ? kb / 8 : kb / 16;
   if (s > s_max) s = s_max;
-  if (s > s_cap) s = s_cap;
   if (s < 1) s = 1;
   if (rem == 0 || s == 1) {
     // data parallel: whole tiles, round robin over the pairs
@@ -758,10 +761,7 @@ cudaError_t launch_bn(const GemmArgs& a, Params p, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   const int max_clusters = n > 0 ? (n < sm_count() / 2 ? n : sm_count() / 2) : 1;
   const int64_t tiles = ((a.M + 2 * BM - 1) / (2 * BM)) * (a.N / BN);
-  // The QKV finisher's epilogue (per-head norm and rotation over the summed
-  // partials) is the heaviest; more than two ranges per tile measured slower.
-  const int s_cap = EPI == static_cast<int>(Epi::kQkv) ? 2 : 1 << 20;
-  const HostSched h = make_sched(tiles, static_cast<int>(a.K / BK), max_clusters, s_cap);
+  const HostSched h = make_sched(tiles, static_cast<int>(a.K / BK), max_clusters);
   const int grid = 2 * h.pairs;
   if (h.sk_units > 0 &&
       (a.sk_partials == nullptr || a.sk_flags == nullptr || grid > a.sk_slots ||
