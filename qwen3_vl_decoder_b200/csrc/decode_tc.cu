@@ -70,10 +70,14 @@ struct DecGemmParams {
   const int32_t* len;    // [B]
 };
 
-__device__ __forceinline__ float dec_row_scale(const DecGemmParams& p, int j) {
+// 1/rms of token j, by the whole warp: from the previous kernel's per-block
+// row sums of squares (the lanes load them at once and add them in a fixed
+// tree), or the precomputed 1/rms.
+__device__ __forceinline__ float dec_row_scale(const DecGemmParams& p, int j, int lane) {
   if (p.rowsq_in != nullptr) {
     float ss = 0.f;
-    for (int t = 0; t < p.rowsq_n; ++t) ss += p.rowsq_in[j * p.rowsq_n + t];
+    for (int t = lane; t < p.rowsq_n; t += 32) ss += p.rowsq_in[j * p.rowsq_n + t];
+    ss = warp_sum(ss);
     return 1.0f / sqrtf(ss / p.rowsq_width + p.eps);
   }
   return p.inv[j];
@@ -86,33 +90,67 @@ __device__ __forceinline__ bool dec_token_valid(const DecGemmParams& p, int j, i
   return slot >= 0 && slot < p.n_seq && row >= 0 && static_cast<int64_t>(row) < p.cap;
 }
 
-// Final epilogue of one token j of row tile `tile`, one warp: lane l holds
-// features l + 32 i (i < 4) of each 128-row block r.
+// The global inputs of one token's epilogue (lane l's features l + 32 i):
+// the 1/rms s (kQkv, kSwiGLU); bias and q/k-norm gain (kQkv) or the
+// residual (kResidual) in a and b; the token's cos/sin pairs (kQkv).
+struct DecEpiIn {
+  float s;
+  float a[4], b[4];
+  float2 cs[2];
+};
+
+// Loads them. Everything it reads is final once griddepcontrol.wait has
+// returned, so an epilogue warp that knows its token does this while the
+// MMAs still run.
 template <int EPI>
-__device__ __forceinline__ void dec_epilogue_token(const DecGemmParams& p, int tile, int j,
-                                                   int lane, float (&v)[2][4]) {
+__device__ __forceinline__ void dec_epilogue_load(const DecGemmParams& p, int tile, int j, int lane,
+                                                  DecEpiIn& in) {
+  const int64_t c0 = int64_t(tile) * 128;
   if constexpr (EPI == static_cast<int>(Epi::kQkv)) {
-    const float s = dec_row_scale(p, j);
-    const int64_t c0 = int64_t(tile) * 128;
+    const bool is_q = tile < p.n_heads, is_k = !is_q && tile < p.n_heads + p.n_kv;
+    const float* gsrc = is_q ? p.q_norm : p.k_norm;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      v[0][i] *= s;
-      if (p.bias != nullptr) v[0][i] += p.bias[c0 + lane + 32 * i];
+      in.a[i] = p.bias != nullptr ? p.bias[c0 + lane + 32 * i] : 0.f;
+      in.b[i] = (is_q || is_k) ? gsrc[lane + 32 * i] : 0.f;
     }
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+      in.cs[i] = (is_q || is_k) ? p.cs[j * 64 + lane + 32 * i] : make_float2(1.f, 0.f);
+    in.s = dec_row_scale(p, j, lane);
+  } else if constexpr (EPI == static_cast<int>(Epi::kResidual)) {
+    const bool ok = dcheck(j < p.B && c0 + 128 <= p.N, p.err, kWhereDbgDecodeStore);
+    const __nv_bfloat16* r = p.resid + int64_t(j) * p.N + c0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) in.a[i] = ok ? bf16_to_f(r[lane + 32 * i]) : 0.f;
+  } else if constexpr (EPI == static_cast<int>(Epi::kSwiGLU)) {
+    in.s = dec_row_scale(p, j, lane);
+  }
+}
+
+// Final epilogue of one token j of row tile `tile`, one warp: lane l holds
+// features l + 32 i (i < 4) of each 128-row block r; `in` holds the loaded
+// inputs of that token.
+template <int EPI>
+__device__ __forceinline__ void dec_epilogue_token(const DecGemmParams& p, int tile, int j,
+                                                   int lane, float (&v)[2][4], const DecEpiIn& in) {
+  if constexpr (EPI == static_cast<int>(Epi::kQkv)) {
+    const int64_t c0 = int64_t(tile) * 128;
     const bool is_q = tile < p.n_heads, is_k = !is_q && tile < p.n_heads + p.n_kv;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[0][i] = v[0][i] * in.s + in.a[i];
     if (is_q || is_k) {
       float ss = 0.f;
 #pragma unroll
       for (int i = 0; i < 4; ++i) ss += v[0][i] * v[0][i];
       ss = warp_sum(ss);
       const float rn = 1.0f / sqrtf(ss * (1.0f / 128.0f) + p.eps);
-      const float* g = is_q ? p.q_norm : p.k_norm;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) v[0][i] *= rn * g[lane + 32 * i];
+      for (int i = 0; i < 4; ++i) v[0][i] *= rn * in.b[i];
       // split-half rotation: feature f pairs with f + 64 (i with i + 2)
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
-        const float2 q = p.cs[j * 64 + lane + 32 * i];
+        const float2 q = in.cs[i];
         const float a = v[0][i], b = v[0][i + 2];
         v[0][i] = a * q.x - b * q.y;
         v[0][i + 2] = a * q.y + b * q.x;
@@ -142,12 +180,11 @@ __device__ __forceinline__ void dec_epilogue_token(const DecGemmParams& p, int t
   } else if constexpr (EPI == static_cast<int>(Epi::kResidual)) {
     const int64_t c0 = int64_t(tile) * 128;
     if (!dcheck(j < p.B && c0 + 128 <= p.N, p.err, kWhereDbgDecodeStore)) return;
-    const __nv_bfloat16* r = p.resid + int64_t(j) * p.N + c0;
     __nv_bfloat16* o = p.out + int64_t(j) * p.N + c0;
     float ss = 0.f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const __nv_bfloat16 ob = __float2bfloat16_rn(bf16_to_f(r[lane + 32 * i]) + v[0][i]);
+      const __nv_bfloat16 ob = __float2bfloat16_rn(in.a[i] + v[0][i]);
       o[lane + 32 * i] = ob;
       const float f = bf16_to_f(ob);
       ss += f * f;
@@ -164,12 +201,11 @@ __device__ __forceinline__ void dec_epilogue_token(const DecGemmParams& p, int t
     for (int i = 0; i < 4; ++i)
       if (lane + 32 * i < left) o[lane + 32 * i] = v[0][i];
   } else {  // kSwiGLU: block 0 = gate rows, block 1 = the matching up rows
-    const float s = dec_row_scale(p, j);
     if (!dcheck(j < p.B && (int64_t(tile) + 1) * 128 <= p.N, p.err, kWhereDbgDecodeStore)) return;
     __nv_bfloat16* o = p.out + int64_t(j) * p.N + int64_t(tile) * 128;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      o[lane + 32 * i] = __float2bfloat16_rn(silu_fast(v[0][i] * s) * (v[1][i] * s));
+      o[lane + 32 * i] = __float2bfloat16_rn(silu_fast(v[0][i] * in.s) * (v[1][i] * in.s));
   }
 }
 
@@ -219,6 +255,9 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   griddep_launch_dependents();
+  // the first token this warp finishes in the split sum below
+  const int pre_j = warp >= 2 ? split + (warp - 2) * p.splits : p.B;
+  DecEpiIn pre{};
 
   if (warp == 0) {
     if (lane == 0) {
@@ -277,8 +316,10 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     __syncwarp();
   } else {
     // epilogue warps: wait for the accumulator (TMEM lanes 32 q .. 32 q + 31
-    // of warp q = warp % 4 are this tile's weight rows, columns are tokens)
+    // of warp q = warp % 4 are this tile's weight rows, columns are tokens),
+    // loading the inputs of this warp's first token meanwhile
     griddep_wait();
+    if (pre_j < p.B) dec_epilogue_load<EPI>(p, tile, pre_j, lane, pre);
     bool ok = true;
     if (lane == 0) ok = mbar_wait(acc_full, 0, p.err, kWhereDecodeEpilogue, abort_flag);
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -338,7 +379,13 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
               for (int i = 0; i < 4; ++i) v[r][i] += w[r][i];
           }
         }
-        dec_epilogue_token<EPI>(p, tile, j0 + jj, lane, v);
+        if (j0 + jj == pre_j) {
+          dec_epilogue_token<EPI>(p, tile, j0 + jj, lane, v, pre);
+        } else {
+          DecEpiIn in;
+          dec_epilogue_load<EPI>(p, tile, j0 + jj, lane, in);
+          dec_epilogue_token<EPI>(p, tile, j0 + jj, lane, v, in);
+        }
       }
     }
     cluster_sync();  // no CTA overwrites or leaves its buffer while another may read it
