@@ -363,22 +363,24 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
       for (int jj = split + e * p.splits; jj < nj; jj += 4 * p.splits) {
         float v[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         const uint32_t own = smem_u32(red + jj * rstride + lane);
+        // every split's values requested before any is added: one DSMEM
+        // round trip, then the sum in split order
+        float w[kDecMaxSplits][R][4];
 #pragma unroll
         for (int sp = 0; sp < kDecMaxSplits; ++sp) {
-          if (sp < p.splits) {
-            const uint32_t ra = map_to_cta(own, static_cast<uint32_t>(sp));
-            float w[2][4];
+          const uint32_t ra = map_to_cta(own, static_cast<uint32_t>(sp < p.splits ? sp : 0));
 #pragma unroll
-            for (int r = 0; r < 2; ++r)
+          for (int r = 0; r < R; ++r)
 #pragma unroll
-              for (int i = 0; i < 4; ++i)
-                w[r][i] = r < R ? ld_dsmem_f32(ra + 4u * (r * 128 + 32 * i)) : 0.f;
-#pragma unroll
-            for (int r = 0; r < 2; ++r)
-#pragma unroll
-              for (int i = 0; i < 4; ++i) v[r][i] += w[r][i];
-          }
+            for (int i = 0; i < 4; ++i)
+              w[sp][r][i] = sp < p.splits ? ld_dsmem_f32(ra + 4u * (r * 128 + 32 * i)) : 0.f;
         }
+#pragma unroll
+        for (int sp = 0; sp < kDecMaxSplits; ++sp)
+#pragma unroll
+          for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) v[r][i] += w[sp][r][i];
         if (j0 + jj == pre_j) {
           dec_epilogue_token<EPI>(p, tile, j0 + jj, lane, v, pre);
         } else {
@@ -450,6 +452,7 @@ struct DecAttnTcParams {
 };
 
 constexpr int kAttnMaxBuf = 3;
+constexpr int kAttnMaxCs = 16;  // most splits of a (b, g) in one cluster
 
 // Byte offset of element (row r, column c) in a 128-byte-swizzled tile of
 // 64-column blocks with `block_bytes` per block (rows of 128 bytes).
@@ -838,17 +841,26 @@ decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tmK,
         for (int idx = static_cast<int>(r) * 128 + t; idx < G * 128; idx += p.cs * 128) {
           const int h = idx >> 7, d = idx & 127;
           const uint32_t base = smem_u32(s_part + h * kAttnRows);
+          // every split's (m, l, o) requested before any is used: one DSMEM
+          // round trip, then the merge in split order
+          float ms[kAttnMaxCs], ls[kAttnMaxCs], os[kAttnMaxCs];
+#pragma unroll
+          for (int sp = 0; sp < kAttnMaxCs; ++sp) {
+            const uint32_t ra = map_to_cta(base, static_cast<uint32_t>(sp < p.cs ? sp : 0));
+            ms[sp] = sp < p.cs ? ld_dsmem_f32(ra + 128 * 4) : -INFINITY;
+            ls[sp] = sp < p.cs ? ld_dsmem_f32(ra + 129 * 4) : 0.f;
+            os[sp] = sp < p.cs ? ld_dsmem_f32(ra + 4u * d) : 0.f;
+          }
           float M = -INFINITY;
-          for (int sp = 0; sp < p.cs; ++sp)
-            M = fmaxf(M, ld_dsmem_f32(map_to_cta(base + 128 * 4, static_cast<uint32_t>(sp))));
+#pragma unroll
+          for (int sp = 0; sp < kAttnMaxCs; ++sp) M = fmaxf(M, ms[sp]);
           float num = 0.f, den = 0.f;
-          for (int sp = 0; sp < p.cs; ++sp) {
-            const uint32_t ra = map_to_cta(base, static_cast<uint32_t>(sp));
-            const float m = ld_dsmem_f32(ra + 128 * 4);
-            if (m == -INFINITY) continue;  // a split without chunks
-            const float w = ex2_approx(m - M);
-            num = fmaf(w, ld_dsmem_f32(ra + 4u * d), num);
-            den = fmaf(w, ld_dsmem_f32(ra + 129 * 4), den);
+#pragma unroll
+          for (int sp = 0; sp < kAttnMaxCs; ++sp) {
+            if (ms[sp] == -INFINITY) continue;  // a split without chunks, or past cs
+            const float w = ex2_approx(ms[sp] - M);
+            num = fmaf(w, os[sp], num);
+            den = fmaf(w, ls[sp], den);
           }
           if (dcheck(int64_t(b) < p.B, p.err, kWhereDbgDecodeStore))
             ob[h * 128 + d] = __float2bfloat16_rn(num / den);
@@ -1103,7 +1115,7 @@ cudaError_t launch_attn_tc_g(const CUtensorMap& tmK, const CUtensorMap& tmV, Dec
     if (e != cudaSuccess) return e;
   }
   int64_t cs = sm_count() / groups;
-  if (cs > 16) cs = 16;
+  if (cs > kAttnMaxCs) cs = kAttnMaxCs;
   if (cs > max_nc) cs = max_nc;
   p.cs = 0;
   for (; cs >= 2; --cs) {
