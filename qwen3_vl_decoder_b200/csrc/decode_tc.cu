@@ -467,7 +467,7 @@ __host__ __device__ constexpr size_t attn_tc_smem_bytes(int nc_pad, int nbuf) {
   return 1024 + size_t(nbuf) * kAttnKV + 2 * kAttnSmall +        // K/V stages, Q
          (nbuf > 1 ? size_t(nbuf) * 2 * kAttnSmall : 0) +         // P (aliases Q if nbuf = 1)
          size_t(2) * G * nc_pad * 4 + size_t(4) * 8 * 4 * 2 +   // merge weights; warp partials
-         size_t(3) * G * 4 + (2 * kDecMaxB + 2) * 4 +           // m, l, den; items
+         size_t(3) * G * 4 + (4 * kDecMaxB + 2) * 4 +           // m, l, den; items, slots, lengths
          size_t(G) * kAttnRows * 4 + 128;                        // cluster partial; barriers
 }
 
@@ -495,7 +495,9 @@ decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tmK,
   int* s_nc = reinterpret_cast<int*>(s_den + G);           // [kDecMaxB] splits per token
   int* s_pref = s_nc + kDecMaxB;                           // [kDecMaxB + 1]
   int* s_last = s_pref + kDecMaxB + 1;
-  float* s_part = reinterpret_cast<float*>(s_last + 1);    // [G][kAttnRows]: o[128], m, l
+  int* s_slot = s_last + 1;                                // [kDecMaxB] seq[b], or -1 if invalid
+  int* s_len = s_slot + kDecMaxB;                          // [kDecMaxB] len[b]
+  float* s_part = reinterpret_cast<float*>(s_len + kDecMaxB);  // [G][kAttnRows]: o[128], m, l
   uint64_t* bars = reinterpret_cast<uint64_t*>(
       (reinterpret_cast<uintptr_t>(s_part + G * kAttnRows) + 7) & ~uintptr_t(7));
   uint64_t* kv_full = bars;                                // [kAttnMaxBuf]
@@ -537,6 +539,8 @@ decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tmK,
     const bool ok = slot >= 0 && slot < p.n_seq && L >= 0 && static_cast<int64_t>(L) < p.cap;
     const int nc = ok ? (L + kAttnCH) / kAttnCH : 0;  // chunks of rows 0..L
     s_nc[b] = p.cs > 0 ? p.cs : (nc < p.nsplit ? nc : p.nsplit);
+    s_slot[b] = ok ? slot : -1;
+    s_len[b] = ok ? L : 0;
   }
   __syncthreads();
   if (warp == 0) {
@@ -578,9 +582,7 @@ decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tmK,
     const int loc = it - s_pref[b];
     g = loc / splits;
     sidx = loc % splits;
-    const int slot = p.seq[b], L = p.len[b];
-    const bool ok = slot >= 0 && slot < p.n_seq && L >= 0 && static_cast<int64_t>(L) < p.cap;
-    const int nc = ok ? (L + kAttnCH) / kAttnCH : 0;
+    const int nc = s_slot[b] >= 0 ? (s_len[b] + kAttnCH) / kAttnCH : 0;
     c0 = static_cast<int>(int64_t(sidx) * nc / splits);
     c1 = static_cast<int>(int64_t(sidx + 1) * nc / splits);
   };
@@ -599,7 +601,7 @@ decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tmK,
     if (l_it >= total) return;
     const int st = n_issued % nbuf;
     uint8_t* dst = s_kv + size_t(st) * kAttnKV;
-    const int32_t y = static_cast<int32_t>(int64_t(p.seq[l_b]) * p.cap + int64_t(l_c) * kAttnCH);
+    const int32_t y = static_cast<int32_t>(int64_t(s_slot[l_b]) * p.cap + int64_t(l_c) * kAttnCH);
     mbar_arrive_expect_tx(kv_full + st, kAttnKV);
     tma_load_2d(dst, &tmK, kv_full + st, l_g * 128, y);
     tma_load_2d(dst + kAttnBlk, &tmK, kv_full + st, l_g * 128 + 64, y);
@@ -633,7 +635,7 @@ decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tmK,
     if (*s_abort && p.cs == 0) break;
     int b, g, c0, c1, splits, s;
     item(it, b, g, c0, c1, splits, s);
-    const int L1 = p.len[b] + 1;
+    const int L1 = s_len[b] + 1;
     float m_run[G], l_run[G], o_run[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) { m_run[h] = -INFINITY; l_run[h] = 0.f; o_run[h] = 0.f; }
@@ -663,7 +665,7 @@ decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tmK,
       const bool has_new = cn >= c && cn < c + nb;
       uint4 kv_new = make_uint4(0, 0, 0, 0);
       if (has_new && t < 32) {
-        const int64_t row = int64_t(p.seq[b]) * p.cap + (L1 - 1);
+        const int64_t row = int64_t(s_slot[b]) * p.cap + (L1 - 1);
         const __nv_bfloat16* src = (t < 16 ? p.kc : p.vc) + row * (int64_t(p.nkv) * 128) + g * 128;
         kv_new = *reinterpret_cast<const uint4*>(src + (t & 15) * 8);
       }
@@ -834,8 +836,7 @@ decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tmK,
         }
       }
       cluster_sync();
-      const int slot = p.seq[b], L = p.len[b];
-      const bool tok_ok = slot >= 0 && slot < p.n_seq && L >= 0 && static_cast<int64_t>(L) < p.cap;
+      const bool tok_ok = s_slot[b] >= 0;
       if (tok_ok && *s_abort == 0) {
         const uint32_t r = cluster_ctarank();
         for (int idx = static_cast<int>(r) * 128 + t; idx < G * 128; idx += p.cs * 128) {
