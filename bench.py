@@ -261,26 +261,33 @@ class E2EPipeline:
     Every step copies its inputs (x, token types, grids) from pinned host
     memory to the device, runs P0..P9, and copies x' back to pinned host
     memory. Uploads, compute and downloads run on three streams with
-    double-buffered device inputs, so step k+1's upload and step k-1's
-    download overlap step k's kernels, as a serving loop would.
+    triple-buffered device inputs, so step k+1's upload and step k-1's
+    download overlap each other and step k's kernels, as a serving loop
+    would (with two buffers, step k+1's upload would have to wait for step
+    k-1's download of the same buffer).
     """
+
+    NBUF = 3
 
     def __init__(self, st, dev):
         self.st = st
         self.s_in = torch.cuda.Stream(dev)
         self.s_out = torch.cuda.Stream(dev)
         self.s_comp = torch.cuda.current_stream(dev)
-        self.x = [st["x"], torch.empty_like(st["x"])]
-        self.tt = [st["tt"], torch.empty_like(st["tt"])]
-        self.g = [st["g"], None if st["g"] is None else torch.empty_like(st["g"])]
-        self.out = [st["out_host"], torch.empty_like(st["out_host"]).pin_memory()]
-        self.in_done = [torch.cuda.Event() for _ in range(2)]
-        self.comp_done = [torch.cuda.Event() for _ in range(2)]
-        self.out_done = [torch.cuda.Event() for _ in range(2)]
-        self.started = [False, False]
+        n = self.NBUF
+        self.x = [st["x"]] + [torch.empty_like(st["x"]) for _ in range(n - 1)]
+        self.tt = [st["tt"]] + [torch.empty_like(st["tt"]) for _ in range(n - 1)]
+        self.g = [st["g"]] + [None if st["g"] is None else torch.empty_like(st["g"])
+                              for _ in range(n - 1)]
+        self.out = [st["out_host"]] + [torch.empty_like(st["out_host"]).pin_memory()
+                                       for _ in range(n - 1)]
+        self.in_done = [torch.cuda.Event() for _ in range(n)]
+        self.comp_done = [torch.cuda.Event() for _ in range(n)]
+        self.out_done = [torch.cuda.Event() for _ in range(n)]
+        self.started = [False] * n
 
     def step(self, k):
-        st, q3, b = self.st, self.st["q3"], k % 2
+        st, q3, b = self.st, self.st["q3"], k % self.NBUF
         with torch.cuda.stream(self.s_in):
             if self.started[b]:
                 self.s_in.wait_event(self.out_done[b])   # x[b] was read by its download
