@@ -583,6 +583,41 @@ def stack_leg(w, dev, steps, warmup, final_norm_reps=50):
     return out
 
 
+def elementwise_leg(dev, hbm, rows=65536, reps=20):
+    """The standalone row-statistic (P2) and final-norm (P10) kernels on a
+    4B-width activation of `rows` rows (335 MB of bf16 at 65536), far larger
+    than one layer call's 21 MB, where launch and ramp latency dominate: the
+    kernels' own bandwidth. Bytes: P2 reads x and writes 1/rms; P10 reads x
+    and the gain and writes x."""
+    import qwen3_vl_decoder_b200 as q3
+    w = syn.Q4B_LAYER
+    cfg = q3.config_of(w)
+    H = w.hidden
+    g = torch.Generator(device=dev).manual_seed(5)
+    x = torch.randn(rows, H, generator=g, device=dev).to(torch.bfloat16)
+    gain = (1 + 0.1 * torch.randn(H, generator=g, device=dev)).to(torch.bfloat16)
+    out = {"rows": rows, "width": H}
+    for name, fn, nb in (("rowstat", lambda: q3.rms_rowstat(cfg, x), 2 * rows * H + 4 * rows),
+                         ("final_norm", lambda: q3.final_norm(cfg, x, gain),
+                          4 * rows * H + 2 * H)):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        t = e0.elapsed_time(e1) / 1e3 / reps
+        out[name] = {"us": 1e6 * t, "bytes": nb,
+                     "roofline": {"bound": "hbm", "achieved": nb / t / 1e9, "peak": hbm,
+                                  "unit": "GB/s", "frac": nb / t / 1e9 / hbm}}
+    q3.check_device()
+    del x
+    torch.cuda.empty_cache()
+    return out
+
+
 def kernel_rooflines(w, stage_ms, peak, peak_name, hbm):
     """Per-kernel algorithmic work over its live stage time."""
     S, H, I = w.seq, w.hidden, w.intermediate
@@ -710,6 +745,7 @@ def main():
         also[syn.Q2B_STACK.name] = stack_leg(syn.Q2B_STACK, dev, steps=10, warmup=3)
         also[syn.Q32B_ENC_1064.name] = stack_leg(syn.Q32B_ENC_1064, dev, steps=5, warmup=2)
         also[syn.Q32B_ENC.name] = stack_leg(syn.Q32B_ENC, dev, steps=3, warmup=1)
+        also["elementwise-4b-width-s65536"] = elementwise_leg(dev, peaks()[2])
         also["context"] = ("the pages time one workload of this path: a 1064-token encode through "
                            "the 32B-shape encoder truncated at layer 50, 29 s (55 s with the "
                            "dequantize-and-host-GEMM arm) on a 28-core AVX2 host with quantized "
