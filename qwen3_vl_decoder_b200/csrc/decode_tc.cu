@@ -410,18 +410,23 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
 //   S^T [128 rows x 16] = K_chunk [128 x 128] . Q^T        (K-major A and B)
 //   O^T [128 dims x 16] = V_chunk^T [128 x 128] . P^T      (V as an MN-major A)
 // K and V arrive by TMA (128-byte swizzle); thread t owns TMEM lane t (cache
-// row t for the softmax, dimension t for the output). An item issues a few
-// hundred instructions per thread (a CUDA-core version took ~1.8k), but runs
-// its chain (load, S, softmax, O) serially, so three CTAs share an SM to
-// overlap one another's chains.
+// row t for the softmax, dimension t for the output).
 //
 // A work item is a contiguous range of 128-row chunks of one (token b, KV
-// head g); the host splits each group into about as many items as fill the
-// CTA slots (one per SM when there are fewer groups than SMs). The chunks of
-// an item merge on the fly in registers (running max m, sum l and o per head,
-// base-2 exponents with log2(e)/sqrt(128) applied to S in fp32). A group with
-// one item writes o / l; otherwise the last item of the group to finish (a
-// ticket counter) merges the items:
+// head g). The chunks of an item merge on the fly in registers (running max
+// m, sum l and o per head, base-2 exponents with log2(e)/sqrt(128) applied to
+// S in fp32). The cached rows below len[b] do not change during a decode
+// call, so each CTA requests its first chunks before waiting for the QKV
+// projection and patches the new row in after the wait. Two forms:
+//   - small batches: the cs splits of a (b, g) are one cluster, one CTA per
+//     SM with a ring of kAttnMaxBuf chunk stages; the chunks in the ring go
+//     through one S / softmax / O pass together, and the cs partials merge
+//     over DSMEM;
+//   - otherwise three CTAs share an SM with one stage each, about one item
+//     per SM; a (b, g) with one item writes o / l, else the last item of the
+//     group to finish (a ticket counter) merges the partials from global
+//     memory.
+// Either merge computes
 //   o = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s,  M = max_s m_s.
 // ---------------------------------------------------------------------------
 constexpr int kAttnCH = 128;    // cache rows per chunk (the MMA's M)
