@@ -82,7 +82,12 @@ def test_prefill_kv_writes_the_layers_k_and_v(w):
     # batches whose items span several 128-row chunks (merged in registers):
     (syn.Q2B_LAYER, [900 + 3 * b for b in range(16)]),  # 4 splits of ~2 chunks per (b, g)
     (syn.Q2B_LAYER, [400 + b for b in range(64)]),      # 1 split of 4 chunks per (b, g)
-], ids=["2b-b4", "4b-b3", "2b-b40", "32b-b2", "2b-b16-multichunk", "2b-b64-multichunk"])
+    # clusters of 2 splits, each walking ~8 chunks through the 3-stage ring in several passes
+    (syn.Q4B_LAYER, [1900 + 37 * b for b in range(9)]),
+    # one CTA slot per item, the last split of a (b, g) merging from global memory
+    (syn.Q4B_LAYER, [700 + 13 * b for b in range(10)]),
+], ids=["2b-b4", "4b-b3", "2b-b40", "32b-b2", "2b-b16-multichunk", "2b-b64-multichunk",
+        "4b-b9-cluster2", "4b-b10-ticket"])
 def test_layer_decode_matches_oracle(w, lens):
     m = q3()
     cfg = m.config_of(w)
