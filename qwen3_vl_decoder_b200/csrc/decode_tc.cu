@@ -472,7 +472,7 @@ __host__ __device__ constexpr size_t attn_tc_smem_bytes(int nc_pad, int nbuf) {
   return 1024 + size_t(nbuf) * kAttnKV + 2 * kAttnSmall +        // K/V stages, Q
          (nbuf > 1 ? size_t(nbuf) * 2 * kAttnSmall : 0) +         // P (aliases Q if nbuf = 1)
          size_t(2) * G * nc_pad * 4 + size_t(4) * 8 * 4 * 2 +   // merge weights; warp partials
-         size_t(3) * G * 4 + (4 * kDecMaxB + 2) * 4 +           // m, l, den; items, slots, lengths
+         size_t(G) * 4 + (4 * kDecMaxB + 2) * 4 +               // den; items, slots, lengths
          size_t(G) * kAttnRows * 4 + 128;                        // cluster partial; barriers
 }
 
@@ -494,9 +494,7 @@ decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tmK,
   float* s_cl = s_w + G * p.nc_pad;                        // [G][nc_pad]
   float* s_wm = s_cl + G * p.nc_pad;                       // [4 warps][8]
   float* s_wl = s_wm + 32;                                 // [4 warps][8]
-  float* s_m = s_wl + 32;
-  float* s_l = s_m + G;
-  float* s_den = s_l + G;
+  float* s_den = s_wl + 32;                                // [G]
   int* s_nc = reinterpret_cast<int*>(s_den + G);           // [kDecMaxB] splits per token
   int* s_pref = s_nc + kDecMaxB;                           // [kDecMaxB + 1]
   int* s_last = s_pref + kDecMaxB + 1;
