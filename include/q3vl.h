@@ -315,7 +315,10 @@ size_t q3vl_decode_workspace_bytes(const q3vl_config* cfg, int32_t B, int64_t ca
  * A seq or len out of range is recorded as the device error Q3VL_ERANGE and
  * that token's output row is left unspecified.
  * ws:  device workspace of >= q3vl_decode_workspace_bytes(cfg, B, cap)
- *      bytes, 256-byte aligned. */
+ *      bytes, 256-byte aligned.
+ * The call starts after all earlier work in `stream`; its attention reads the
+ * cached rows 0..len[b]-1 while the projection before it still runs, so no
+ * other stream may write those rows during the call. */
 int q3vl_layer_decode(const q3vl_config* cfg, const q3vl_layer* layer, void* x, int32_t B,
                       const int32_t* pos, const q3vl_kv_cache* kv, const int32_t* seq,
                       const int32_t* len, void* ws, size_t ws_bytes, q3vl_stream stream);
