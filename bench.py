@@ -123,9 +123,12 @@ def traffic_for_current_kernel():
 class ClockSampler:
     """SM clock, power and clock-event reasons sampled during the timed region.
 
-    A thread polls NVML (read-only queries) every few milliseconds between
+    A child process (a fresh interpreter, not a fork of this CUDA process)
+    polls NVML with read-only queries every half millisecond between
     __enter__ and __exit__, so even a timed region of a few tens of
-    milliseconds gets samples. Without NVML it falls back to nvidia-smi.
+    milliseconds gets samples: a thread of this process would wait for the
+    interpreter lock while the timed loop launches and synchronises. Without
+    NVML it falls back to nvidia-smi.
     """
     REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
                ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4),
@@ -133,48 +136,62 @@ class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    POLLER = (
+        "import signal, sys, time\n"
+        "import pynvml\n"
+        "signal.signal(signal.SIGTERM, lambda *a: (sys.stdout.flush(), sys.exit(0)))\n"
+        "pynvml.nvmlInit()\n"
+        "key, period = sys.argv[1], float(sys.argv[2])\n"
+        "h = (pynvml.nvmlDeviceGetHandleByUUID(key) if key.startswith('GPU-')\n"
+        "     else pynvml.nvmlDeviceGetHandleByIndex(int(key)))\n"
+        "smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)\n"
+        "print('ready', flush=True)\n"
+        "k, pw = 0, 0.0\n"
+        "while True:\n"
+        "    sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)\n"
+        "    mask = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)\n"
+        "    if k % 8 == 0:\n"
+        "        pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1e3\n"
+        "    print(f'{sm},{smax},{mask},{pw}')\n"
+        "    k += 1\n"
+        "    time.sleep(period)\n")
 
-    def __init__(self, dev, period_s=0.002):
+    def __init__(self, dev, period_s=0.0005):
         self.dev = dev
         self.period = period_s
         self.samples = []      # (sm_mhz, sm_max_mhz, reason mask, power W)
         self.source = None
         self.proc = None
+        self.lines = []
         self.out = ""
 
-    def _nvml_handle(self):
-        import pynvml
-        pynvml.nvmlInit()
+    def _key(self):
         try:
             uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
-            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(
-                uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            return uuid if uuid.startswith("GPU-") else "GPU-" + uuid
         except Exception:
-            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.dev.index or 0)
-
-    def _poll(self):
-        nv, h = self.nv, self.h
-        smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
-        while not self.stop.is_set():
-            try:
-                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
-                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
-                pw = nv.nvmlDeviceGetPowerUsage(h) / 1e3
-                self.samples.append((float(sm), float(smax), int(mask), pw))
-            except Exception:
-                break
-            self.stop.wait(self.period)
+            return str(self.dev.index or 0)
 
     def __enter__(self):
         import threading
-        self.stop = threading.Event()
-        self.thread = None
+        self.reader = None
         try:
-            self.nv, self.h = self._nvml_handle()
+            import pynvml  # noqa: F401  (the child needs it)
+            self.proc = subprocess.Popen(
+                [sys.executable, "-c", self.POLLER, self._key(), str(self.period)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            if self.proc.stdout.readline().strip() != "ready":
+                raise RuntimeError("NVML poller did not start")
             self.source = "nvml"
-            self.thread = threading.Thread(target=self._poll, daemon=True)
-            self.thread.start()
+            # drain the pipe so the child never blocks on a full buffer
+            self.reader = threading.Thread(
+                target=lambda: self.lines.extend(self.proc.stdout), daemon=True)
+            self.reader.start()
         except Exception:
+            if self.proc is not None:
+                self.proc.kill()
+                self.proc.wait()
+            self.proc = None
             self.source = "nvidia-smi"
             try:
                 self.proc = subprocess.Popen(
@@ -187,26 +204,40 @@ class ClockSampler:
         return self
 
     def __exit__(self, *a):
-        if self.thread is not None:
-            self.stop.set()
-            self.thread.join(timeout=2)
-        if self.proc is not None:
+        if self.proc is None:
+            return
+        if self.source == "nvml":
             self.proc.terminate()
             try:
-                self.out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                self.out, _ = self.proc.communicate()
-            for r in (self.out or "").strip().splitlines():
-                f = r.split(",")
-                if len(f) < 9:
-                    continue
-                try:
-                    mask = sum(bit for (n, bit), v in zip(self.REASONS[:4], f[5:9])
-                               if v.strip() not in ("", "[N/A]") and "Not" not in v)
-                    self.samples.append((float(f[1]), float(f[2]), mask, float(f[3] or 0)))
-                except ValueError:
-                    continue
+                self.proc.wait()
+            self.reader.join(timeout=5)
+            for r in self.lines:
+                f = r.strip().split(",")
+                if len(f) == 4:
+                    try:
+                        self.samples.append((float(f[0]), float(f[1]), int(f[2]), float(f[3])))
+                    except ValueError:
+                        continue
+            return
+        self.proc.terminate()
+        try:
+            self.out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            self.out, _ = self.proc.communicate()
+        for r in (self.out or "").strip().splitlines():
+            f = r.split(",")
+            if len(f) < 9:
+                continue
+            try:
+                mask = sum(bit for (n, bit), v in zip(self.REASONS[:4], f[5:9])
+                           if v.strip() not in ("", "[N/A]") and "Not" not in v)
+                self.samples.append((float(f[1]), float(f[2]), mask, float(f[3] or 0)))
+            except ValueError:
+                continue
 
     def summary(self):
         if not self.samples:
