@@ -468,7 +468,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             // B already requested; stage `stage` is in its first use
             tma_load_2d_pair(smA + stage * C::kABytes, &tmA, fb, kb * BK, m0);
           } else {
-            if (!mbar_wait(empty + stage, ph ^ 1, p.err, kWhereGemmProducer, abort_flag)) {
+            if (!mbar_wait<true>(empty + stage, ph ^ 1, p.err, kWhereGemmProducer, abort_flag)) {
               ok = false;
               break;
             }
@@ -490,7 +490,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       if (lead_cta)
         for (int s = 0; s < S; ++s)
           if (issued & (1u << s))
-            mbar_wait(full + s, (last_ph >> s) & 1u, p.err, kWhereGemmDrain, nullptr);
+            mbar_wait<true>(full + s, (last_ph >> s) & 1u, p.err, kWhereGemmDrain, nullptr);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -504,12 +504,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         bool ok = true;
         while (ok && it.next(w)) {
           const int buf = acc_i & 1;
-          if (!mbar_wait(tempty + buf, ((acc_i >> 1) & 1) ^ 1, p.err, kWhereGemmMma, abort_flag))
+          if (!mbar_wait<true>(tempty + buf, ((acc_i >> 1) & 1) ^ 1, p.err, kWhereGemmMma, abort_flag))
             break;
           tc_fence_after();
           const uint32_t d = tmem_base + buf * BN;
           for (int kb = w.kb0; kb < w.kb1; ++kb) {
-            if (!mbar_wait(full + stage, ph, p.err, kWhereGemmMma, abort_flag)) { ok = false; break; }
+            if (!mbar_wait<true>(full + stage, ph, p.err, kWhereGemmMma, abort_flag)) { ok = false; break; }
             tc_fence_after();
             const uint32_t a0 = smem_u32(smA + stage * C::kABytes);
             const uint32_t b0 = smem_u32(smB + stage * C::kBBytes);
@@ -528,7 +528,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         // All issued MMAs complete before either CTA releases its TMEM.
         umma_commit_pair(drain, 0x3);
       }
-      mbar_wait(drain, 0, p.err, kWhereGemmDrain, nullptr);
+      mbar_wait<true>(drain, 0, p.err, kWhereGemmDrain, nullptr);
     }
   } else {
     griddep_wait();  // the epilogue reads and writes this layer's activations
@@ -566,9 +566,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           tma_load_2d(tile + b * 16384, &tmRes, res_full, static_cast<int32_t>(n0 + 64 * b),
                       static_cast<int32_t>(row0));
       }
-      bool ok = mbar_wait(tfull + buf, (acc_i >> 1) & 1, p.err, kWhereGemmEpilogue, abort_flag);
+      bool ok = mbar_wait<true>(tfull + buf, (acc_i >> 1) & 1, p.err, kWhereGemmEpilogue, abort_flag);
       if (need_res) {
-        ok = ok && mbar_wait(res_full, res_ph, p.err, kWhereGemmEpilogue, abort_flag);
+        ok = ok && mbar_wait<true>(res_full, res_ph, p.err, kWhereGemmEpilogue, abort_flag);
         res_ph ^= 1;
       }
       if (!ok) *abort_flag = 1;

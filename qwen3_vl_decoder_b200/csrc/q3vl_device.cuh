@@ -98,18 +98,39 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The same with a suspend-time hint: the thread may sleep up to
+// kTryWaitHintNs in the instruction (it resumes when the phase completes), so
+// a waiting role takes fewer issue slots from the warps doing the work.
+// Measured on the 4B layer: the GEMMs 1-4% faster, the attention (whose
+// softmax warps wait for each score tile) 3% slower, decode unchanged.
+constexpr uint32_t kTryWaitHintNs = 10000;
+__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "n"(kTryWaitHintNs)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase of `bar` with the given parity to complete. Gives up
 // after kWaitLimitNs (or as soon as another role of the block raised
 // *abort), records Q3VL_ETIMEOUT and returns false. Never spins forever.
+// kSuspend: poll with the suspend-time hint.
+template <bool kSuspend = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* err,
                                           int32_t where, volatile int* abort,
                                           uint64_t limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait(a, parity)) return true;
+  auto try_wait = [&]() { return kSuspend ? mbar_try_wait_hint(a, parity) : mbar_try_wait(a, parity); };
+  if (try_wait()) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(a, parity)) return true;
+      if (try_wait()) return true;
     if (abort != nullptr && *abort) return false;
     if (globaltimer_ns() - t0 > limit_ns) {
       record_error(err, Q3VL_ETIMEOUT, where);
