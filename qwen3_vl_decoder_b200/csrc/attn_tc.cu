@@ -512,23 +512,30 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, 128, false, true);
+      // The issuing thread shares its SM sub-partition with two softmax
+      // warps, and each head's chain waits for its 16 products to be issued:
+      // the descriptors are formed once and advanced by constant offsets
+      // (the start-address field holds the address / 16; every address stays
+      // below 256 KB, so the sum never carries out of the field).
+      const uint64_t dq0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(smem_u32(sV), kBlockBytes, 1024);
       auto issue_s = [&](int x, int t) {
-        const uint32_t q0 = smem_u32(sQ + x * kTileBytes);
-        const uint32_t k0 = smem_u32(sK + (t & 1) * kTileBytes);
+        const uint64_t dq = dq0 + static_cast<uint64_t>((x * kTileBytes) >> 4);
+        const uint64_t dk = dk0 + static_cast<uint64_t>(((t & 1) * kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kBlockBytes + (kk & 3) * 32;
-          umma_bf16_ss(tmem + x * 128, sdesc_sw128(q0 + off, 16, 1024),
-                       sdesc_sw128(k0 + off, 16, 1024), idesc_s, kk > 0);
+          const uint64_t off = ((kk >> 2) * kBlockBytes + (kk & 3) * 32) >> 4;
+          umma_bf16_ss(tmem + x * 128, dq + off, dk + off, idesc_s, kk > 0);
         }
         umma_commit(s_full + x);
       };
       auto issue_pv = [&](int x, int j, int t) {
-        const uint32_t v0 = smem_u32(sV + (t & 1) * kTileBytes);
+        const uint64_t dv = dv0 + static_cast<uint64_t>(((t & 1) * kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_bf16_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8,
-                       sdesc_sw128(v0 + kk * 2048, kBlockBytes, 1024), idesc_o, (j | kk) != 0);
+          umma_bf16_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, dv + ((kk * 2048) >> 4), idesc_o,
+                       (j | kk) != 0);
       };
       bool ok = true;
       int t0 = 0;  // this CTA's tile index of the item's first key tile
