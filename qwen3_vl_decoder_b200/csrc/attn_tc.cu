@@ -555,6 +555,9 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
           const int t = t0 + j, s = t & 1;
           const bool more = j + 1 < n_kv;
           if (!mbar_wait(v_full + s, (t >> 1) & 1, p.err, kWhereAttnMma, abort_flag)) { ok = false; break; }
+          // the next K tile has usually landed by now: checking it here keeps
+          // the wait off the stretch between P_A and S_A(j+1)
+          bool k_next = !more || mbar_try_wait(smem_u32(k_full + (s ^ 1)), ((t + 1) >> 1) & 1);
           if (!mbar_wait(p_full + 0, t & 1, p.err, kWhereAttnMma, abort_flag)) { ok = false; break; }
           // the first P V of an item overwrites O: the previous item's O_A
           // must have been read out
@@ -563,11 +566,13 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
           tc_fence_after();
           issue_pv(0, j, t);
           if (more) {
-            if (!mbar_wait(k_full + (s ^ 1), ((t + 1) >> 1) & 1, p.err, kWhereAttnMma, abort_flag)) {
-              ok = false;
-              break;
+            if (!k_next) {
+              if (!mbar_wait(k_full + (s ^ 1), ((t + 1) >> 1) & 1, p.err, kWhereAttnMma, abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
             }
-            tc_fence_after();
             issue_s(0, t + 1);
           }
           if (!mbar_wait(p_full + 1, t & 1, p.err, kWhereAttnMma, abort_flag)) { ok = false; break; }
@@ -620,11 +625,14 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
         const bool grow = m_new > m + kRescaleLog2;
         const float alpha = grow ? ex2_approx(m - m_new) : 1.0f;
         if (grow) m = m_new;
+        // the warp's rescale decision before the exponentials, so nothing
+        // but the stores is left between them and the arrival
+        const bool rescale = j > 0 && __any_sync(0xffffffffu, grow);
         // P = 2^(s*scale - m) as bf16 into the first 64 columns of S
         const float rs = diag ? exp_regs<true, kPoly>(sr, tS, r, sc, m)
                               : exp_regs<false, kPoly>(sr, tS, r, sc, m);
         l = l * alpha + rs;
-        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        if (rescale) {
           // O_X(j-1) is complete: S_X(j) was issued after P_X(j-1) V(j-1).
 #pragma unroll 1
           for (int c4 = 0; c4 < 4; ++c4) {
