@@ -86,3 +86,36 @@ def test_random_prompts_with_videos():
 def test_single_token():
     pos, nxt = _run([0], [])
     assert pos.cpu().tolist() == [[0], [0], [0]] and nxt == 1
+
+
+@pytest.mark.parametrize("cut", [4, 7, 127, 4095])
+def test_run_broken_at_a_thread_warp_or_chunk_boundary(cut):
+    # one image of n tokens whose run is broken by a text token at `cut`; the
+    # token after it starts a thread's four tokens (7 -> 8), a warp's (127 ->
+    # 128) or the next 4096-token chunk (4095 -> 4096)
+    n = cut + 9
+    types = [1] * cut + [0] + [1] * (n - cut)
+    with pytest.raises(q3().Q3VLError) as e:
+        _run(types, [(1, 1, n)])
+    assert e.value.code == -3
+
+
+def test_unaligned_token_types():
+    # a token-type array that does not start on a 4-byte boundary takes the
+    # byte loads; same positions as the oracle
+    rng = np.random.default_rng(9)
+    types, grids = [], []
+    while len(types) < 5000:
+        types += [0] * int(rng.integers(0, 20))
+        r, c = int(rng.integers(1, 20)), int(rng.integers(1, 20))
+        types += [1] * (r * c)
+        grids.append((1, r, c))
+    buf = torch.zeros(len(types) + 1, dtype=torch.uint8, device="cuda")
+    buf[1:] = torch.tensor(types, dtype=torch.uint8, device="cuda")
+    tt = buf[1:]
+    assert tt.data_ptr() % 4 == 1
+    gd = torch.tensor(grids, dtype=torch.int32, device="cuda").reshape(-1, 3)
+    pos, nxt = q3().mrope_positions(tt, gd)
+    ref, ref_next = O.mrope_positions_tokens(types, grids)
+    assert np.array_equal(pos.cpu().numpy(), ref)
+    assert nxt == ref_next
