@@ -383,7 +383,11 @@ __device__ __forceinline__ float exp_regs(const uint32_t* sr, uint32_t tS, int r
 }
 
 constexpr int kThreads2 = 320;
-constexpr size_t kSmem2 = 1024 + 6 * size_t(kTileBytes) + 256;  // Q_A, Q_B, K[2], V[2]
+// Q_A, Q_B, K[2], V[2], barriers, and 4 KB per softmax warp to stage its
+// output rows for coalesced stores
+constexpr int kStageBytes2 = 32 * 128;
+constexpr size_t kSmem2 = 1024 + 6 * size_t(kTileBytes) + 256 + 8 * size_t(kStageBytes2);
+static_assert(kSmem2 <= 232448, "shared memory budget");
 constexpr float kRescaleLog2 = 8.0f;
 // Pairs of every 16 whose exponentials run on the FMA pipe. Measured on the
 // 4B layer at S = 4096: 0 -> 137.7 us, 2 -> 141.8, 4 -> 135.7, 6 -> 145.9
@@ -423,6 +427,7 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
   uint64_t* o_free = bars + 16;  // [2] per head
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint8_t* s_out = smem + 6 * kTileBytes + 256;  // [8 softmax warps][32 rows x 128 B]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pairs = p.nh / 2;
@@ -607,7 +612,6 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
     int t = 0;  // this CTA's running tile index
     for (int ii = 0, k = item_of(0); ok && k >= 0; k = item_of(++ii)) {
       const int qt = p.num_qt - 1 - k / pairs, h0 = 2 * (k % pairs);
-      const int64_t qpos = int64_t(qt) * kTile + r;
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j <= qt; ++j, ++t) {
         ok = mbar_wait(s_full + x, t & 1, p.err, kWhereAttnSoftmax, abort_flag);
@@ -653,7 +657,6 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
       const float inv_l = 1.0f / l;
-      __nv_bfloat16* dst = p.o + qpos * p.ldo + (h0 + x) * 128;
       uint32_t o[4][32];
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(tO + 32 * c4, o[c4]);
@@ -661,18 +664,33 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
       // O is in registers: the next item's first P V may overwrite it
       tc_fence_before();
       mbar_arrive(o_free + x);
-      if (qpos < p.S && dcheck(((h0 + x) + 1) * 128 <= p.ldo, p.err, kWhereDbgAttnStore)) {
+      // The warp's 32 rows go out through shared memory, 64 columns at a
+      // time: each thread stages its row's 128 bytes (16-byte units swizzled
+      // by row), then every store instruction writes four whole 128-byte row
+      // segments instead of 16 bytes of 32 rows 8 KB apart.
+      uint8_t* stg = s_out + (warp - 2) * kStageBytes2;
+      const bool cols_ok = dcheck(((h0 + x) + 1) * 128 <= p.ldo, p.err, kWhereDbgAttnStore);
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c4);
+      for (int hf = 0; hf < 2; ++hf) {
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
-            d4[u] = make_uint4(
-                pack_bf16x2(__uint_as_float(o[c4][8 * u]) * inv_l, __uint_as_float(o[c4][8 * u + 1]) * inv_l),
-                pack_bf16x2(__uint_as_float(o[c4][8 * u + 2]) * inv_l, __uint_as_float(o[c4][8 * u + 3]) * inv_l),
-                pack_bf16x2(__uint_as_float(o[c4][8 * u + 4]) * inv_l, __uint_as_float(o[c4][8 * u + 5]) * inv_l),
-                pack_bf16x2(__uint_as_float(o[c4][8 * u + 6]) * inv_l, __uint_as_float(o[c4][8 * u + 7]) * inv_l));
+        for (int u = 0; u < 8; ++u) {
+          const uint32_t* ov = o[2 * hf + (u >> 2)] + 8 * (u & 3);
+          *reinterpret_cast<uint4*>(stg + lane * 128 + ((u ^ (lane & 7)) << 4)) = make_uint4(
+              pack_bf16x2(__uint_as_float(ov[0]) * inv_l, __uint_as_float(ov[1]) * inv_l),
+              pack_bf16x2(__uint_as_float(ov[2]) * inv_l, __uint_as_float(ov[3]) * inv_l),
+              pack_bf16x2(__uint_as_float(ov[4]) * inv_l, __uint_as_float(ov[5]) * inv_l),
+              pack_bf16x2(__uint_as_float(ov[6]) * inv_l, __uint_as_float(ov[7]) * inv_l));
         }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int rr = 4 * i + (lane >> 3), u = lane & 7;
+          const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * 128 + ((u ^ (rr & 7)) << 4));
+          const int64_t row = int64_t(qt) * kTile + quarter * 32 + rr;
+          if (row < p.S && cols_ok)
+            *reinterpret_cast<uint4*>(p.o + row * p.ldo + (h0 + x) * 128 + 64 * hf + 8 * u) = v;
+        }
+        __syncwarp();
       }
     }
   }
