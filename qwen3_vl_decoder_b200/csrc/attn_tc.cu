@@ -383,8 +383,8 @@ __device__ __forceinline__ float exp_regs(const uint32_t* sr, uint32_t tS, int r
 }
 
 constexpr int kThreads2 = 320;
-// Q_A, Q_B, K[2], V[2], barriers, and 4 KB per softmax warp to stage its
-// output rows for coalesced stores
+// Q_A, Q_B, K[2], V[2], 4 KB per softmax warp for the output box it stores
+// by TMA, and the barriers
 constexpr int kStageBytes2 = 32 * 128;
 constexpr size_t kSmem2 = 1024 + 6 * size_t(kTileBytes) + 256 + 8 * size_t(kStageBytes2);
 static_assert(kSmem2 <= 232448, "shared memory budget");
@@ -407,13 +407,15 @@ constexpr int kPolyPairs = 4;
 // per CTA tile index t (a tile = one key tile of one item).
 template <int kPoly>
 __global__ void __launch_bounds__(kThreads2, 1)
-attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
+attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ CUtensorMap tmo,
+                Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint8_t* sQ = smem;                   // [2] heads
   uint8_t* sK = smem + 2 * kTileBytes;  // [2] stages
   uint8_t* sV = smem + 4 * kTileBytes;  // [2] stages
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 6 * kTileBytes);
+  uint8_t* s_out = smem + 6 * kTileBytes;  // [8 softmax warps][32 rows x 128 B], 128-byte swizzle
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_out + 8 * kStageBytes2);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;   // [2]
   uint64_t* k_empty = bars + 3;  // [2]
@@ -427,7 +429,6 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
   uint64_t* o_free = bars + 16;  // [2] per head
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  uint8_t* s_out = smem + 6 * kTileBytes + 256;  // [8 softmax warps][32 rows x 128 B]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pairs = p.nh / 2;
@@ -453,6 +454,7 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm);
+    tma_prefetch_desc(&tmo);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -664,14 +666,20 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
       // O is in registers: the next item's first P V may overwrite it
       tc_fence_before();
       mbar_arrive(o_free + x);
-      // The warp's 32 rows go out through shared memory, 64 columns at a
-      // time: each thread stages its row's 128 bytes (16-byte units swizzled
-      // by row), then every store instruction writes four whole 128-byte row
-      // segments instead of 16 bytes of 32 rows 8 KB apart.
+      // The warp's 32 rows go out by TMA, 64 columns at a time: each thread
+      // writes its row's 128 bytes into the warp's staging box in the
+      // 128-byte swizzle the tensor map expects, and one lane issues the
+      // bulk store. The warps move on to the next item at once; the stores of
+      // all CTAs, which finish their items at about the same time, drain in
+      // the background (as 16-byte stores into 32 rows 8 KB apart they held
+      // the softmax warps ~4,000 cycles per item).
       uint8_t* stg = s_out + (warp - 2) * kStageBytes2;
       const bool cols_ok = dcheck(((h0 + x) + 1) * 128 <= p.ldo, p.err, kWhereDbgAttnStore);
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
+        // the box is free once the previous bulk store has read it
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const uint32_t* ov = o[2 * hf + (u >> 2)] + 8 * (u & 3);
@@ -681,19 +689,19 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, Params p) {
               pack_bf16x2(__uint_as_float(ov[4]) * inv_l, __uint_as_float(ov[5]) * inv_l),
               pack_bf16x2(__uint_as_float(ov[6]) * inv_l, __uint_as_float(ov[7]) * inv_l));
         }
+        fence_proxy_async_smem();
         __syncwarp();
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int rr = 4 * i + (lane >> 3), u = lane & 7;
-          const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * 128 + ((u ^ (rr & 7)) << 4));
-          const int64_t row = int64_t(qt) * kTile + quarter * 32 + rr;
-          if (row < p.S && cols_ok)
-            *reinterpret_cast<uint4*>(p.o + row * p.ldo + (h0 + x) * 128 + 64 * hf + 8 * u) = v;
+        // rows past S are clipped by the tensor map; a box wholly past it
+        // is not issued
+        const int32_t y0 = qt * kTile + quarter * 32;
+        if (lane == 0 && cols_ok && y0 < p.S) {
+          tma_store_2d(&tmo, stg, (h0 + x) * 128 + 64 * hf, y0);
+          bulk_commit_group();
         }
-        __syncwarp();
       }
     }
   }
+  if (warp >= 2 && lane == 0) bulk_wait_all();  // this warp's output stores complete
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -722,12 +730,15 @@ cudaError_t launch_attention_tc(const q3vl_config& c, const void* qkv, int64_t S
   p.err = device_error_ptr();
   if ((p.nh / p.nkv) % 2 == 0) {
     // two query heads of one KV group per CTA
+    // the output, [S, nh * 128] with row stride ldo, in 64-column x 32-row boxes
+    CUtensorMap tmo;
+    if (!make_tmap_bf16(&tmo, o, S, q_dim(c), p.ldo, 64, 32)) return cudaErrorInvalidValue;
     auto kern = attn2_tc_kernel<kPolyPairs>;
     cudaError_t e = smem_attr_at_least(reinterpret_cast<const void*>(kern), kSmem2);
     if (e != cudaSuccess) return e;
     const int64_t items = int64_t(p.num_qt) * (p.nh / 2);
     const unsigned grid = static_cast<unsigned>(items < sm_count() ? items : sm_count());
-    e = launch_pdl_plain(kern, dim3(grid), dim3(kThreads2), kSmem2, st, tm, p);
+    e = launch_pdl_plain(kern, dim3(grid), dim3(kThreads2), kSmem2, st, tm, tmo, p);
     if (e != cudaSuccess) return e;
     return counted_launch(1);
   }
