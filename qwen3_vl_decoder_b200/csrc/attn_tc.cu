@@ -423,11 +423,11 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ 
   uint64_t* v_empty = bars + 7;  // [2]
   uint64_t* s_full = bars + 9;   // [2] per head
   uint64_t* p_full = bars + 11;  // [2] per head
-  uint64_t* o_final = bars + 13;
-  uint64_t* drain = bars + 14;
-  uint64_t* q_empty = bars + 15;
-  uint64_t* o_free = bars + 16;  // [2] per head
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
+  uint64_t* o_final = bars + 13;  // [2] per head
+  uint64_t* drain = bars + 15;
+  uint64_t* q_empty = bars + 16;
+  uint64_t* o_free = bars + 17;  // [2] per head
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -448,8 +448,8 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ 
       mbar_init(v_full + s, 1); mbar_init(v_empty + s, 1);
       mbar_init(s_full + s, 1); mbar_init(p_full + s, 128);
       mbar_init(o_free + s, 128);
+      mbar_init(o_final + s, 1);
     }
-    mbar_init(o_final, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -546,18 +546,22 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ 
       };
       bool ok = true;
       int t0 = 0;  // this CTA's tile index of the item's first key tile
+      // The first item's first score products; every later item's follow
+      // the previous item's last P V of the same head (below).
+      if (item_of(0) >= 0) {
+        ok = mbar_wait(q_full, 0, p.err, kWhereAttnMma, abort_flag) &&
+             mbar_wait(k_full + 0, 0, p.err, kWhereAttnMma, abort_flag);
+        if (ok) {
+          tc_fence_after();
+          issue_s(0, 0);
+          issue_s(1, 0);
+          umma_commit(k_empty + 0);
+          if (p.num_qt - item_of(0) / pairs == 1) umma_commit(q_empty);
+        }
+      }
       for (int ii = 0, k = item_of(0); ok && k >= 0; k = item_of(++ii)) {
         const int n_kv = p.num_qt - k / pairs;
-        ok = mbar_wait(q_full, ii & 1, p.err, kWhereAttnMma, abort_flag) &&
-             mbar_wait(k_full + (t0 & 1), (t0 >> 1) & 1, p.err, kWhereAttnMma, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        // S_X(0) overwrites P_X of the previous item's last tile only after
-        // that tile's P V, issued before it, has read it (in-order execution)
-        issue_s(0, t0);
-        issue_s(1, t0);
-        umma_commit(k_empty + (t0 & 1));
-        if (n_kv == 1) umma_commit(q_empty);
+        const int kn = item_of(ii + 1), tn = t0 + n_kv;  // the next item and its first tile
         for (int j = 0; j < n_kv; ++j) {
           const int t = t0 + j, s = t & 1;
           const bool more = j + 1 < n_kv;
@@ -581,6 +585,21 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ 
               tc_fence_after();
             }
             issue_s(0, t + 1);
+          } else {
+            // head A's O is complete once this P V is; the next item's
+            // first S_A follows it (S_A overwrites P_A only after this P V,
+            // issued before it, has read P_A: in-order execution), so head
+            // A's softmax warps start the next item while head B finishes
+            umma_commit(o_final + 0);
+            if (kn >= 0) {
+              if (!mbar_wait(q_full, (ii + 1) & 1, p.err, kWhereAttnMma, abort_flag) ||
+                  !mbar_wait(k_full + (tn & 1), (tn >> 1) & 1, p.err, kWhereAttnMma, abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              issue_s(0, tn);
+            }
           }
           if (!mbar_wait(p_full + 1, t & 1, p.err, kWhereAttnMma, abort_flag)) { ok = false; break; }
           if (j == 0 && ii > 0 &&
@@ -592,9 +611,15 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ 
             issue_s(1, t + 1);
             umma_commit(k_empty + (s ^ 1));
             if (j + 2 == n_kv) umma_commit(q_empty);  // the item's last S products
+          } else {
+            umma_commit(o_final + 1);
+            if (kn >= 0) {
+              issue_s(1, tn);
+              umma_commit(k_empty + (tn & 1));
+              if (p.num_qt - kn / pairs == 1) umma_commit(q_empty);  // the next item's only tile
+            }
           }
         }
-        umma_commit(o_final);
         t0 += n_kv;
       }
       if (!ok) *abort_flag = 1;
@@ -655,7 +680,7 @@ attn2_tc_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ 
         mbar_arrive(p_full + x);
       }
       if (!ok) break;
-      ok = mbar_wait(o_final, ii & 1, p.err, kWhereAttnSoftmax, abort_flag);
+      ok = mbar_wait(o_final + x, ii & 1, p.err, kWhereAttnSoftmax, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
       const float inv_l = 1.0f / l;
