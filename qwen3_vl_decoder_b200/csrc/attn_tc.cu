@@ -399,10 +399,12 @@ constexpr int kPolyPairs = 4;
 // CTA c takes items c, 2G-1-c, 2G+c, 4G-1-c, ... (G CTAs, a snake that
 // evens out the causal tile counts). Across items the pipeline keeps going:
 // the TMA warp loads the next item's Q as soon as the last S of the current
-// item has read Q, the MMA warp issues the next item's first S products
-// behind the current item's last P V once that Q and the first K tile have
-// arrived, and only the next item's first P V waits for the softmax warps to
-// have read the finished O out of TMEM.
+// item has read Q; the MMA warp issues each head's first S product of the
+// next item right behind that head's last P V of the current item (once that
+// Q and the first K tile have arrived) and signals the head's finished O on a
+// barrier of its own, so one head's softmax warps write their output and go
+// on while the other head finishes; only the next item's first P V of a head
+// waits for that head's softmax warps to have read its O out of TMEM.
 // Barrier phases run on counters across items: per CTA item index ii and
 // per CTA tile index t (a tile = one key tile of one item).
 template <int kPoly>
