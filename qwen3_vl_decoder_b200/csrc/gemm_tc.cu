@@ -70,7 +70,8 @@ struct Params {
   int32_t* err;
   // schedule over pair tiles (see WorkIter)
   int64_t dp_tiles, sk_units;
-  int sk_pairs;   // pairs 0 .. sk_pairs-1 share the stream-K units
+  int sk_pairs;   // pairs sk_first .. sk_first+sk_pairs-1 share the stream-K units
+  int sk_first;
   int kb_per_tile;
   int m_fastest;  // tile order: 1 = M index fastest (A stays in L2), 0 = N fastest (B stays)
   // stream-K scratch: one fp32 128 x BN partial tile and one flag per CTA
@@ -90,8 +91,8 @@ struct Params {
 //   tiles [0, dp_tiles): data parallel; pair c takes tiles c, c + G, ... over
 //     their whole K range;
 //   tiles [dp_tiles, T): stream-K; their U = (T - dp_tiles) * KB k-block
-//     units are cut into Gs = sk_pairs equal contiguous ranges, pair c < Gs
-//     taking units [c U / Gs, (c + 1) U / Gs).
+//     units are cut into Gs = sk_pairs equal contiguous ranges, pair
+//     sk_first + i (i < Gs) taking units [i U / Gs, (i + 1) U / Gs).
 // A stream-K tile split across pairs is finished by the pair holding its
 // first k-block, which reaches it last (at the end of its stream-K range).
 // The pairs holding its later k-blocks reach them first (at the start of
@@ -112,9 +113,12 @@ struct WorkIter {
   int KB;
   __device__ WorkIter(const Params& p, int c, int G)
       : dp_t(c), dp_tiles(p.dp_tiles), stride(G),
-        u(c < p.sk_pairs ? p.sk_units * c / p.sk_pairs : 0),
-        u1(c < p.sk_pairs ? p.sk_units * (c + 1) / p.sk_pairs : 0), sk_base(p.dp_tiles),
+        u(in_sk(p, c) ? p.sk_units * (c - p.sk_first) / p.sk_pairs : 0),
+        u1(in_sk(p, c) ? p.sk_units * (c - p.sk_first + 1) / p.sk_pairs : 0), sk_base(p.dp_tiles),
         KB(p.kb_per_tile) {}
+  __device__ static bool in_sk(const Params& p, int c) {
+    return c >= p.sk_first && c < p.sk_first + p.sk_pairs;
+  }
   __device__ bool next(Work& w) {
     if (u < u1) {
       const int64_t t = u / KB;
@@ -605,7 +609,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         if (w.role == kFinisher) {
           // contributors: the pairs owning k-blocks [kb1, KB) of this tile
           const int64_t t_rel = w.tile - p.dp_tiles;
-          const int c_last = sk_owner((t_rel + 1) * p.kb_per_tile - 1, p.sk_units, p.sk_pairs);
+          const int c_last =
+              p.sk_first + sk_owner((t_rel + 1) * p.kb_per_tile - 1, p.sk_units, p.sk_pairs);
           const int first = 2 * (c + 1) + static_cast<int>(rank);
           part = p.sk_partials + static_cast<size_t>(first) * slot_floats;
           n_part = c_last - c;
@@ -773,6 +778,12 @@ cudaError_t launch_bn(const GemmArgs& a, Params p, cudaStream_t st) {
   p.kb_per_tile = static_cast<int>(a.K / BK);
   // keep the smaller operand resident in L2 while the larger one streams
   p.m_fastest = a.M <= a.N ? 1 : 0;
+  // The QKV GEMM gives its stream-K ranges to the last pairs: their last
+  // data-parallel tiles are V columns (N runs slowest in its tile order),
+  // whose epilogue is the short one, so the pairs with the extra range do not
+  // also end on a q/k tile's norm and rotation.
+  p.sk_first = (EPI == static_cast<int>(Epi::kQkv) && h.sk_units > 0 && p.m_fastest)
+                   ? h.pairs - h.sk_pairs : 0;
   e = launch_pdl_plain(kern, dim3(grid), dim3(kThreads), C::kSmem, st, tmA, tmB, tmOut, tmRes, p);
   if (e != cudaSuccess) return e;
   return counted_launch(1);
